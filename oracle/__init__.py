@@ -1,0 +1,292 @@
+"""CPU oracle for the Token Sparse Attention prefill path (TEST INFRASTRUCTURE).
+
+This package is test infrastructure, not product code.  Only the test suite,
+``__graft_entry__.smoke()`` and the ``cpu_baseline`` / ``--impl reference``
+legs of ``bench.py`` may import it.  The CUDA path never calls it, shares no
+code with it, and must fail loudly rather than fall back to it.
+
+It is a plain, slow, fp64 restatement of the method as the pages describe it,
+step by step, with numpy library primitives (matmul, exp, sort, cumsum) as
+the only building blocks.  Source of the method (cited below as [GS]): the
+gist.science summary page "Token Sparse Attention: Efficient Long-Context
+Inference with Interleaved Token Selection" (arXiv 2602.03216), section
+"2. Metodologia", sub-sections "Arquitectura Central" (compress, attend,
+decompress per head) and "Cobertura Dinamica de Tokens" (proxy scoring,
+budget, per-head selection).  The abstract pages with the same title
+(chatpaper.ai, icml.cc poster 65647, fugumt.com) state the same
+compress / attend / decompress scheme in summary form.
+
+Readings taken where the page is silent (each is also pinned by a test):
+  * "recent queries" = the last w query positions; the proxy map is causal
+    (window row at position i sees keys j <= i) and uses the attention's
+    own scale 1/sqrt(d) (fp32 value, widened).
+  * importance of key j = sum over the w window rows of the row-normalised
+    proxy weights (the "vertical" sum); computed in fp64, rounded once to
+    fp32 -- the fp32 score is the interface value both sides agree on.
+  * coverage mass is measured exactly: q_j = ceil(score_j * 2^40) as int64,
+    Q = sum q_j, threshold T = floor(tau * Q) in fp64 (tau is fp32).
+    Tokens are taken in ascending q order; the pruned count p_h is the
+    largest p whose first-p prefix sum stays <= T (the token that would
+    push the pruned mass past tau is kept).  k_h = L - p_h.
+  * the "global budget" is per sequence: k_b = max over heads of k_h.
+  * per-head top-k: the k_b indices with the largest fp32 score, equal
+    scores broken toward the smaller index, emitted in ascending order.
+  * compressed causality: compressed row i attends compressed keys j <= i;
+    since indices ascend, this is the original causal order.
+  * GQA: selection per Q head h; K and V rows come from KV head h // G.
+  * scatter: a zero L x d output per head; row S_h[i] receives row i of
+    the compressed output; every other row is exactly zero.
+
+Every function here is pinned in ``tests/test_oracle_pins.py`` against brute
+force, closed forms, hand-derived fixtures (``tests/golden``) and an
+independent library routine (torch's fp64 scaled-dot-product attention).
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from workloads import bf16_bits_to_f64
+
+TWO_POW_40 = float(2 ** 40)
+
+
+def default_scale(d: int) -> float:
+    """Softmax scale: the fp32 value of 1/sqrt(d), widened to fp64."""
+    return float(np.float32(1.0) / np.sqrt(np.float32(d)))
+
+
+def _f64(x: np.ndarray) -> np.ndarray:
+    if x.dtype == np.uint16:
+        return bf16_bits_to_f64(x)
+    return np.asarray(x, dtype=np.float64)
+
+
+# ---------------------------------------------------------------------------
+# Step 1: proxy attention map of the recent queries, summed per key column.
+# [GS] "Cobertura Dinamica de Tokens", scoring bullet.
+# ---------------------------------------------------------------------------
+def proxy_scores_head(q_window: np.ndarray, k_head: np.ndarray, L: int, scale: float,
+                      return_f64: bool = False):
+    """Importance of every key of one head.
+
+    q_window: [w, d] queries at positions L-w .. L-1; k_head: [L, d].
+    Row r (position i = L-w+r) of the proxy map is the softmax over keys
+    j <= i of scale * (q_i . k_j); the importance of key j is the sum of
+    column j over the w rows.
+    """
+    qw = _f64(q_window)
+    kh = _f64(k_head)
+    w = qw.shape[0]
+    x = (qw @ kh.T) * scale                                  # [w, L]
+    pos = np.arange(L - w, L)[:, None]
+    x = np.where(np.arange(L)[None, :] <= pos, x, -np.inf)   # causal proxy map
+    m = x.max(axis=1, keepdims=True)
+    e = np.exp(x - m)
+    p = e / e.sum(axis=1, keepdims=True)                     # row softmax
+    s64 = p.sum(axis=0)                                      # vertical sum
+    s32 = s64.astype(np.float32)
+    return (s32, s64) if return_f64 else s32
+
+
+def proxy_scores(q, k, w: int, scale: float | None = None, return_f64: bool = False):
+    """Scores [B, Hq, L] (fp32) for bf16 inputs q [B,Hq,L,d], k [B,Hkv,L,d]."""
+    B, Hq, L, d = q.shape
+    Hkv = k.shape[1]
+    G = Hq // Hkv
+    if scale is None:
+        scale = default_scale(d)
+    out = np.empty((B, Hq, L), dtype=np.float32)
+    out64 = np.empty((B, Hq, L), dtype=np.float64) if return_f64 else None
+    for b in range(B):
+        for h in range(Hq):
+            r = proxy_scores_head(q[b, h, L - w:], k[b, h // G], L, scale, return_f64)
+            if return_f64:
+                out[b, h], out64[b, h] = r
+            else:
+                out[b, h] = r
+    return (out, out64) if return_f64 else out
+
+
+# ---------------------------------------------------------------------------
+# Step 2: Dynamic Token Coverage budget.
+# [GS] "Cobertura Dinamica de Tokens", budget bullet and per-head bullet.
+# ---------------------------------------------------------------------------
+def quantise_mass(scores: np.ndarray) -> np.ndarray:
+    """Exact fixed-point mass: q = ceil(score * 2^40) as int64 (score >= 0)."""
+    return np.ceil(np.asarray(scores, dtype=np.float32).astype(np.float64) * TWO_POW_40).astype(np.int64)
+
+
+def coverage_threshold(qv: np.ndarray, tau: float) -> np.ndarray:
+    """T = floor(tau * sum(q)) with tau as fp32 widened to fp64."""
+    total = qv.sum(axis=-1)
+    return np.floor(np.float64(np.float32(tau)) * total.astype(np.float64)).astype(np.int64)
+
+
+def pruned_count_head(scores_head: np.ndarray, tau: float) -> int:
+    """Largest p such that the p least important tokens carry mass <= T."""
+    qv = quantise_mass(scores_head)
+    T = int(coverage_threshold(qv, tau))
+    cum = np.cumsum(np.sort(qv))            # ascending importance
+    return int(np.count_nonzero(cum <= T))  # cum is non-decreasing
+
+
+def coverage_budget(scores: np.ndarray, tau: float):
+    """Per-head keep counts k_h = L - p_h [B,Hq] and per-sequence k_b [B]."""
+    B, Hq, L = scores.shape
+    k_head = np.empty((B, Hq), dtype=np.int32)
+    for b in range(B):
+        for h in range(Hq):
+            k_head[b, h] = L - pruned_count_head(scores[b, h], tau)
+    k_seq = k_head.max(axis=1).astype(np.int32)   # global budget of the sequence
+    return k_head, k_seq
+
+
+# ---------------------------------------------------------------------------
+# Step 3: per-head top-k selection, ascending indices.
+# [GS] "Cobertura Dinamica de Tokens", per-head selection bullet, and
+# "Arquitectura Central", compression step.
+# ---------------------------------------------------------------------------
+def select_head(scores_head: np.ndarray, k: int) -> np.ndarray:
+    L = scores_head.shape[0]
+    s = np.asarray(scores_head, dtype=np.float32).astype(np.float64)
+    order = np.lexsort((np.arange(L), -s))     # score descending, index ascending
+    return np.sort(order[:k]).astype(np.int32)
+
+
+def select_topk(scores: np.ndarray, k_seq: np.ndarray) -> np.ndarray:
+    """idx [B,Hq,L] int32: first k_b entries are S_h ascending, the rest -1."""
+    B, Hq, L = scores.shape
+    idx = np.full((B, Hq, L), -1, dtype=np.int32)
+    for b in range(B):
+        for h in range(Hq):
+            kb = int(k_seq[b])
+            idx[b, h, :kb] = select_head(scores[b, h], kb)
+    return idx
+
+
+# ---------------------------------------------------------------------------
+# Step 4: gather into dense compressed tensors.  [GS] "Arquitectura Central".
+# ---------------------------------------------------------------------------
+def gather_qkv(q, k, v, idx, k_seq):
+    """Compressed copies (same dtype as the inputs), rows >= k_b left zero."""
+    B, Hq, L, d = q.shape
+    G = Hq // k.shape[1]
+    qc = np.zeros_like(q)
+    kc = np.zeros((B, Hq, L, d), dtype=k.dtype)
+    vc = np.zeros((B, Hq, L, d), dtype=v.dtype)
+    for b in range(B):
+        kb = int(k_seq[b])
+        for h in range(Hq):
+            s = idx[b, h, :kb]
+            qc[b, h, :kb] = q[b, h, s]
+            kc[b, h, :kb] = k[b, h // G, s]
+            vc[b, h, :kb] = v[b, h // G, s]
+    return qc, kc, vc
+
+
+# ---------------------------------------------------------------------------
+# Step 5: causal attention over the compressed set.  [GS] "Arquitectura
+# Central": the compressed tensors are attended by an ordinary dense kernel.
+# ---------------------------------------------------------------------------
+def attention_rows(qc: np.ndarray, kc: np.ndarray, vc: np.ndarray, rows, scale: float,
+                   chunk: int = 1024) -> np.ndarray:
+    """Causal softmax attention for the listed rows of one head (fp64).
+
+    Row i: o_i = sum_{j<=i} softmax_j(scale * q_i . k_j) v_j.
+    Rows are evaluated independently; ``chunk`` only bounds memory.
+    """
+    rows = np.asarray(rows, dtype=np.int64)
+    out = np.empty((rows.shape[0], vc.shape[-1]), dtype=np.float64)
+    for c0 in range(0, rows.shape[0], chunk):
+        r = rows[c0:c0 + chunk]
+        n = int(r.max()) + 1
+        qf = _f64(qc[r])
+        kf = _f64(kc[:n])
+        vf = _f64(vc[:n])
+        x = (qf @ kf.T) * scale
+        x = np.where(np.arange(n)[None, :] <= r[:, None], x, -np.inf)
+        m = x.max(axis=1, keepdims=True)
+        e = np.exp(x - m)
+        out[c0:c0 + chunk] = (e @ vf) / e.sum(axis=1, keepdims=True)
+    return out
+
+
+def compressed_attention(qc, kc, vc, k_seq, scale: float | None = None) -> np.ndarray:
+    """O_hat [B,Hq,L,d] fp64; rows >= k_b are zero."""
+    B, Hq, L, d = qc.shape
+    if scale is None:
+        scale = default_scale(d)
+    oc = np.zeros((B, Hq, L, d), dtype=np.float64)
+    for b in range(B):
+        kb = int(k_seq[b])
+        for h in range(Hq):
+            oc[b, h, :kb] = attention_rows(qc[b, h, :kb], kc[b, h, :kb], vc[b, h, :kb],
+                                           np.arange(kb), scale)
+    return oc
+
+
+def dense_causal_attention(q, k, v, scale: float | None = None) -> np.ndarray:
+    """Dense causal GQA attention [B,Hq,L,d] fp64: the same row definition on
+    the full sequence (the identity selection)."""
+    B, Hq, L, d = q.shape
+    G = Hq // k.shape[1]
+    if scale is None:
+        scale = default_scale(d)
+    o = np.empty((B, Hq, L, d), dtype=np.float64)
+    for b in range(B):
+        for h in range(Hq):
+            o[b, h] = attention_rows(q[b, h], k[b, h // G], v[b, h // G], np.arange(L), scale)
+    return o
+
+
+# ---------------------------------------------------------------------------
+# Step 6: scatter back into a zero-initialised full-length output.
+# [GS] "Arquitectura Central", decompression step.
+# ---------------------------------------------------------------------------
+def scatter(oc: np.ndarray, idx: np.ndarray, k_seq: np.ndarray, L: int) -> np.ndarray:
+    B, Hq, _, d = oc.shape
+    o = np.zeros((B, Hq, L, d), dtype=oc.dtype)
+    for b in range(B):
+        kb = int(k_seq[b])
+        for h in range(Hq):
+            o[b, h, idx[b, h, :kb]] = oc[b, h, :kb]
+    return o
+
+
+# ---------------------------------------------------------------------------
+# The whole path, step by step.
+# ---------------------------------------------------------------------------
+def forward(q, k, v, w: int, tau: float, scale: float | None = None) -> dict:
+    """Scores -> budget -> selection -> gather -> attention -> scatter."""
+    B, Hq, L, d = q.shape
+    if scale is None:
+        scale = default_scale(d)
+    scores = proxy_scores(q, k, w, scale)
+    k_head, k_seq = coverage_budget(scores, tau)
+    idx = select_topk(scores, k_seq)
+    qc, kc, vc = gather_qkv(q, k, v, idx, k_seq)
+    oc = compressed_attention(qc, kc, vc, k_seq, scale)
+    o = scatter(oc, idx, k_seq, L)
+    return dict(scores=scores, k_head=k_head, k_seq=k_seq, idx=idx, oc=oc, o=o)
+
+
+def output_rows(q, k, v, idx, k_seq, b: int, h: int, orig_rows, scale: float | None = None):
+    """Final output rows (original positions) of head (b, h), computed one by
+    one from a given selection: zero if the position is not selected, else the
+    compressed attention row.  Used to check large workloads by sampling."""
+    B, Hq, L, d = q.shape
+    G = Hq // k.shape[1]
+    if scale is None:
+        scale = default_scale(d)
+    kb = int(k_seq[b])
+    s = np.asarray(idx[b, h, :kb], dtype=np.int64)
+    orig_rows = np.asarray(orig_rows, dtype=np.int64)
+    pos = np.searchsorted(s, orig_rows)
+    hit = (pos < kb) & (s[np.minimum(pos, kb - 1)] == orig_rows)
+    out = np.zeros((orig_rows.shape[0], d), dtype=np.float64)
+    if hit.any():
+        cpos = pos[hit]
+        n = int(cpos.max()) + 1
+        sel = s[:n]
+        out[hit] = attention_rows(q[b, h][sel], k[b, h // G][sel], v[b, h // G][sel], cpos, scale)
+    return out
