@@ -1,0 +1,380 @@
+"""Benchmark of the Token Sparse Attention prefill path on B200.
+
+One step = one pass of the whole hot path (proxy scores, coverage budget,
+per-head top-k, gather, compressed causal attention, scatter) over one
+synthetic 128K-token prefill (32 query / 8 KV heads, d = 128, w = 128,
+tau = 0.05), through the C ABI.  Metric: effective TFLOP/s = dense causal
+attention FLOPs of the workload / TSA time (the speedup over our dense causal
+kernel on the same tensors is reported beside it).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--tau T] [--impl reference]
+
+With --gpus N > 1 (under torchrun) every rank runs its own sequence: the
+units shard across ranks with no data-path collective (weak scaling); the
+step time is the max over ranks.  --impl reference times the CPU oracle on a
+bounded sample of the same workload on the host cores (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "Token-sparse prefill attention ms and effective TFLOP/s at 128K vs dense; % BF16/HBM roofline"
+UNIT = "TFLOP/s (effective: dense causal attention FLOPs / TSA time)"
+DEFAULT_WORKLOAD = "c4_L128K_gqa"
+KERNELS_PER_FORWARD = 8  # score x3, budget, select, gather, attend, scatter
+
+
+def dense_flops(wl) -> float:
+    return float(wl.B) * wl.Hq * 2.0 * wl.d * wl.L * (wl.L + 1)
+
+
+def compressed_flops(wl, k_seq) -> float:
+    return float(sum(wl.Hq * 2.0 * wl.d * int(k) * (int(k) + 1) for k in k_seq))
+
+
+def peaks() -> dict:
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            m = json.load(f)
+        return {"hbm_gbs": m["hbm_gbs"], "bf16": m["bf16_tflops"], "bf16_sustained": m["bf16_tflops_sustained"],
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during timing."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self) -> dict:
+        rows = []
+        if self.path and os.path.exists(self.path):
+            with open(self.path) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) >= 9:
+                        rows.append(parts)
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        load = [s for s in sm if mx and s > 0.5 * max(mx)] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- oracle leg
+def oracle_sample(wl, tau: float, rows: int = 48) -> dict:
+    """Time the CPU oracle on a bounded sample of the workload and scale it to
+    the whole step: steps 1-4 and 6 for one head at full length, step 5 for
+    the `rows` most expensive compressed rows of that head."""
+    import oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([t.get("num_threads", 1) for t in threadpool_info()] or [1])
+    except Exception:  # pragma: no cover
+        cores = 1
+    q, k, v = W.generate(wl.with_(B=1, Hq=1, Hkv=1))
+    L, d = wl.L, wl.d
+    scale = O.default_scale(d)
+    t0 = time.perf_counter()
+    s32 = O.proxy_scores_head(q[0, 0, L - wl.w:], k[0, 0], L, scale)
+    kh = L - O.pruned_count_head(s32, tau)
+    sel = O.select_head(s32, kh)
+    qc, kc, vc = q[0, 0][sel], k[0, 0][sel], v[0, 0][sel]
+    t1 = time.perf_counter()
+    r = np.arange(kh - rows, kh)
+    oc = O.attention_rows(qc, kc, vc, r, scale)
+    t2 = time.perf_counter()
+    full = np.zeros((L, d))
+    full[sel[r]] = oc
+    t3 = time.perf_counter()
+    per_head_fixed = (t1 - t0) + (t3 - t2)
+    sample_pairs = float(np.sum(r + 1))
+    head_pairs = kh * (kh + 1) / 2.0
+    t_full = wl.B * wl.Hq * (per_head_fixed + (t2 - t1) * head_pairs / sample_pairs)
+    return {"seconds_full_step_est": t_full, "cores": cores, "sample_seconds": t3 - t0,
+            "k_head": int(kh),
+            "sample": (f"steps 1-4,6 for head (0,0) at L={L}, step 5 for its last {rows} compressed rows "
+                       f"(of k={kh}); scaled by head count and by causal pair count to the full step")}
+
+
+def run_reference(args, wl, rank: int) -> int:
+    if rank != 0:
+        return 0
+    for _ in range(args.warmup):
+        oracle_sample(wl, args.tau)
+    runs = [oracle_sample(wl, args.tau) for _ in range(args.steps)]
+    t = statistics.median(r["seconds_full_step_est"] for r in runs)
+    value = dense_flops(wl) / t / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "L": wl.L, "d": wl.d,
+                   "w": wl.w, "tau": args.tau},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": runs[0]["cores"], "kind": "oracle",
+                         "sample": runs[0]["sample"]},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- GPU leg
+def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
+    import torch
+    import token_sparse_attention_tsa_b200 as T
+
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist_mod
+        dist = dist_mod
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    T.load()
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    def max_over_ranks(x: float) -> float:
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    # inputs: this rank's own sequence (seed offset by rank)
+    wl_r = wl.with_(seed=wl.seed + 1000 * rank)
+    qh, kh, vh = W.generate(wl_r)
+    pin = [torch.from_numpy(x).view(torch.bfloat16).pin_memory() for x in (qh, kh, vh)]
+    q, k, v = [x.to(dev, non_blocking=True) for x in pin]
+    o = torch.empty_like(q)
+    p = T.params(wl.B, wl.Hq, wl.Hkv, wl.L, wl.d, wl.w, args.tau)
+    ws = T.new_workspace(p, full=True, device=dev)
+    scores = torch.empty((wl.B, wl.Hq, wl.L), dtype=torch.float32, device=dev)
+    idx = torch.empty((wl.B, wl.Hq, wl.L), dtype=torch.int32, device=dev)
+    k_seq = torch.empty((wl.B,), dtype=torch.int32, device=dev)
+    k_head = torch.empty((wl.B, wl.Hq), dtype=torch.int32, device=dev)
+    shape = (wl.B, wl.Hq, wl.L, wl.d)
+    qc, kc, vc, oc = (torch.empty(shape, dtype=torch.bfloat16, device=dev) for _ in range(4))
+    torch.cuda.synchronize()
+
+    def forward():
+        T.tsa_forward(p, q, k, v, o, ws, scores, idx, k_seq)
+
+    stage_names = ["score", "budget", "select", "gather", "attend", "scatter"]
+
+    def staged(evs):
+        evs[0].record(stream)
+        T.tsa_score(p, q, k, scores, ws)
+        evs[1].record(stream)
+        T.tsa_budget(p, scores, k_head, k_seq, ws)
+        evs[2].record(stream)
+        T.tsa_select(p, scores, k_seq, idx, ws)
+        evs[3].record(stream)
+        T.tsa_gather_qkv(p, q, k, v, idx, k_seq, qc, kc, vc, ws)
+        evs[4].record(stream)
+        T.tsa_attend(p, qc, kc, vc, k_seq, oc, None, ws)
+        evs[5].record(stream)
+        T.tsa_scatter(p, oc, idx, k_seq, o, ws)
+        evs[6].record(stream)
+
+    def timed(fn, n):
+        barrier()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        return max_over_ranks(a.elapsed_time(b) / n)
+
+    for _ in range(args.warmup):
+        forward()
+    torch.cuda.synchronize()
+
+    # ---- headline: tsa_forward, inputs resident in HBM (all > L2)
+    with ClockSampler(local_rank) as clk:
+        ms = timed(forward, args.steps)
+    clocks = clk.summary()
+    ks = k_seq.cpu().numpy().tolist()
+
+    # ---- per-stage breakdown (same kernels, one ABI call per stage)
+    per_stage = {n: [] for n in stage_names}
+    for it in range(args.warmup + args.steps):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(7)]
+        barrier()
+        staged(evs)
+        torch.cuda.synchronize()
+        if it >= args.warmup:
+            for i, n in enumerate(stage_names):
+                per_stage[n].append(evs[i].elapsed_time(evs[i + 1]))
+    stage_ms = {n: max_over_ranks(statistics.mean(v)) for n, v in per_stage.items()}
+
+    # ---- dense baselines on the same tensors
+    od = torch.empty_like(q)
+    dense_ms = timed(lambda: T.tsa_attend_dense(p, q, k, v, od, None, ws), max(2, args.steps // 2))
+    sdpa_ms = None
+    try:
+        sdpa = torch.nn.functional.scaled_dot_product_attention
+        sdpa(q, k, v, is_causal=True, enable_gqa=True)
+        sdpa_ms = timed(lambda: sdpa(q, k, v, is_causal=True, enable_gqa=True), 2)
+    except Exception:  # library baseline is optional context
+        sdpa_ms = None
+
+    # ---- end to end: pinned host inputs -> device -> tsa_forward -> host output
+    o_host = torch.empty(shape, dtype=torch.bfloat16).pin_memory()
+
+    def e2e_step():
+        q.copy_(pin[0], non_blocking=True)
+        k.copy_(pin[1], non_blocking=True)
+        v.copy_(pin[2], non_blocking=True)
+        T.tsa_forward(p, q, k, v, o, ws, scores, idx, k_seq)
+        o_host.copy_(o, non_blocking=True)
+
+    e2e_step()
+    e2e_ms = timed(e2e_step, max(2, args.steps // 2))
+    h2d = sum(x.numel() * x.element_size() for x in pin)
+    d2h = o_host.numel() * o_host.element_size()
+
+    status, flags = T.get_device_status(ws)
+    if status != 0:
+        print(json.dumps({"error": f"device status {status} flags {flags}"}), file=sys.stderr)
+        return 3
+
+    # ---- roofline of the dominant kernel (attention: a dense contraction)
+    pk = peaks()
+    cflops = compressed_flops(wl, ks)
+    attn_ms = stage_ms["attend"]
+    achieved = cflops / (attn_ms * 1e-3) / 1e12
+    roof = {"bound": "tensor", "kernel": "attend_kernel<128>", "achieved": achieved,
+            "peak": pk["bf16_sustained"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_sustained"],
+            "traffic": None,
+            "peak_note": f"bf16_tflops_sustained of {pk['source']} peaks (kernel timed inside a long step)"}
+    hbm = pk["hbm_gbs"]
+    tok = wl.B * wl.Hq * wl.L
+    kept = sum(ks) * wl.Hq
+    stage_bytes = {
+        "gather": kept * wl.d * 2 * 3 * 2,                      # 3 rows read + 3 written
+        "scatter": tok * wl.d * 2 + kept * wl.d * 2,            # full write + kept rows read
+        "score": 2 * wl.B * wl.Hkv * wl.L * wl.d * 2 + tok * 4,  # two K passes + scores
+    }
+    stage_roof = {n: {"GB/s": b / (stage_ms[n] * 1e-3) / 1e9, "frac_hbm": b / (stage_ms[n] * 1e-3) / 1e9 / hbm}
+                  for n, b in stage_bytes.items()}
+
+    value = world * dense_flops(wl) / (ms * 1e-3) / 1e12
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        s = oracle_sample(wl, args.tau)
+        cpu = {"value": dense_flops(wl) / s["seconds_full_step_est"] / 1e12, "unit": UNIT, "cores": s["cores"],
+               "kind": "oracle", "sample": s["sample"], "sample_seconds": s["sample_seconds"]}
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "L": wl.L, "d": wl.d, "w": wl.w,
+                   "tau": args.tau, "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "l2": "inputs larger than L2 (Q 1 GiB, K/V 256 MiB each)"},
+        "k_seq": ks, "keep_fraction": [x / wl.L for x in ks],
+        "dense_ms": dense_ms, "speedup_vs_dense": dense_ms / ms, "sdpa_dense_ms": sdpa_ms,
+        "effective_tflops": dense_flops(wl) / (ms * 1e-3) / 1e12,
+        "achieved_tflops": cflops / (ms * 1e-3) / 1e12,
+        "stage_ms": stage_ms, "stage_hbm": stage_roof,
+        "overhead_frac": (sum(stage_ms.values()) - attn_ms) / attn_ms,
+        "roofline": roof, "cpu_baseline": cpu,
+        "e2e": {"value": world * dense_flops(wl) / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": KERNELS_PER_FORWARD * args.steps, "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main() -> int:
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--tau", type=float, default=None)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
+    ap.add_argument("--impl", default="tsa", choices=["tsa", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    wl = W.WORKLOADS[args.workload]
+    if args.tau is None:
+        args.tau = wl.tau
+    wl = wl.with_(tau=args.tau)
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, wl, rank)
+    return run_gpu(args, wl, rank, world, local_rank)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,183 @@
+/*
+ * tsa.h -- C ABI of the Token Sparse Attention prefill path on NVIDIA B200
+ * (sm_100a).
+ *
+ * Method source, cited below as [GS]: the gist.science summary page
+ * "Token Sparse Attention: Efficient Long-Context Inference with Interleaved
+ * Token Selection" (arXiv 2602.03216), section 2 "Metodologia", with its
+ * sub-sections "Arquitectura Central" (per-head compression of Q, K, V into
+ * dense shorter tensors, ordinary attention on them, decompression of the
+ * output into a zero-initialised full-length tensor) and "Cobertura Dinamica
+ * de Tokens" (proxy scoring of recent queries against all keys, a coverage
+ * budget from the ascending importance order, per-head top-k selection).
+ * The abstract pages with the same title (chatpaper.ai, icml.cc poster 65647,
+ * fugumt.com) describe the same compress / attend / decompress scheme.
+ *
+ * Notation: B sequences, Hq query heads, Hkv key/value heads, G = Hq/Hkv,
+ * KV head of query head h is h / G (consecutive grouping), L tokens per
+ * sequence, d head dimension, w proxy window, tau coverage threshold,
+ * k_b keep budget of sequence b, S_h ascending index set of head h.
+ *
+ * Layouts (all row-major, contiguous, little-endian):
+ *   q        bf16 [B, Hq,  L, d]      k, v   bf16 [B, Hkv, L, d]
+ *   o        bf16 [B, Hq,  L, d]      scores fp32 [B, Hq, L]
+ *   idx      int32 [B, Hq, L]: entries [0, k_b) hold S_h ascending, the rest -1
+ *   k_head   int32 [B, Hq]            k_seq  int32 [B]
+ *   qc, kc, vc, oc  bf16 [B, Hq, L, d]: compressed tensors, capacity L rows
+ *            per head, rows [0, k_b) valid (K and V are gathered per query
+ *            head, so a GQA group's heads each get their own compressed copy).
+ *   lse      fp32 [B, Hq, L] (optional): natural-log sum of exp of the
+ *            scaled logits of each valid compressed row.
+ *
+ * Conventions shared by every call:
+ *   - Pointers named q, k, v, o, scores, idx, k_head, k_seq, qc, kc, vc, oc,
+ *     lse and ws are DEVICE pointers on the current CUDA device.  The caller
+ *     owns every buffer; the library allocates and frees nothing and keeps no
+ *     state besides per-device cached attributes.
+ *   - Tensor pointers must be 16-byte aligned; ws must be 256-byte aligned.
+ *   - stream is a cudaStream_t (NULL = legacy default stream).  Every call is
+ *     asynchronous on it and never synchronises the host, except
+ *     tsa_get_device_status.  No call reads k_b back to the host: compressed
+ *     buffers are sized at capacity L and kernels read k_seq on the device.
+ *   - Argument errors are detected on the host and returned before any work
+ *     is enqueued (TSA_ERR_INVALID_ARG, TSA_ERR_UNSUPPORTED,
+ *     TSA_ERR_WORKSPACE).  A failed launch returns TSA_ERR_CUDA.
+ *   - Errors found by kernels (non-finite scores, an index outside [0, L), a
+ *     pipeline wait that ran past its time limit) are OR-ed into the device
+ *     status word at the start of ws; read it with tsa_get_device_status.
+ *     Kernels never trap; on such an error they finish or return early.
+ *   - Supported: d in {64, 128}; Hq % Hkv == 0; 1 <= w <= min(L, 4096);
+ *     0 <= tau < 1; L <= 2^22; B * Hq * L < 2^31.
+ */
+#ifndef TSA_H_
+#define TSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define TSA_ABI_VERSION 1
+
+typedef enum tsa_status {
+  TSA_OK = 0,
+  TSA_ERR_INVALID_ARG = 1,  /* null pointer, bad shape, misaligned pointer  */
+  TSA_ERR_UNSUPPORTED = 2,  /* valid but unsupported (e.g. d = 96)           */
+  TSA_ERR_WORKSPACE = 3,    /* workspace missing or smaller than required    */
+  TSA_ERR_CUDA = 4,         /* a CUDA runtime/driver call or launch failed   */
+  TSA_ERR_NONFINITE = 5,    /* device status: a score was NaN or infinite    */
+  TSA_ERR_TIMEOUT = 6,      /* device status: a pipeline wait timed out      */
+  TSA_ERR_BAD_INDEX = 7     /* device status: an index was outside [0, L)    */
+} tsa_status;
+
+/* Bits of the device status word (first 4 bytes of ws). */
+#define TSA_DEVFLAG_NONFINITE 0x1u
+#define TSA_DEVFLAG_TIMEOUT 0x2u
+#define TSA_DEVFLAG_BAD_INDEX 0x4u
+
+typedef struct tsa_params {
+  int32_t B, Hq, Hkv, L, d;
+  int32_t w;            /* proxy window: the last w query positions          */
+  float tau;            /* coverage threshold, 0 <= tau < 1                  */
+  float softmax_scale;  /* 0 selects 1/sqrt(d) (fp32)                        */
+  uint32_t flags;       /* reserved, must be 0                               */
+  uint32_t timeout_ms;  /* limit of one pipeline wait; 0 selects 2000 ms     */
+} tsa_params;
+
+/* Version of this ABI (TSA_ABI_VERSION of the built library). */
+int32_t tsa_abi_version(void);
+
+/* Human-readable name of a status code.  Never NULL. */
+const char* tsa_status_string(tsa_status s);
+
+/* Host-only validation of p (the same checks every call makes). */
+tsa_status tsa_check_params(const tsa_params* p);
+
+/* Workspace bytes needed by tsa_forward (covers every stage call too). */
+tsa_status tsa_workspace_size(const tsa_params* p, size_t* bytes);
+
+/* Workspace bytes needed by the single-stage calls below (status word and
+ * the proxy-score row statistics; much smaller than tsa_workspace_size). */
+tsa_status tsa_stage_workspace_size(const tsa_params* p, size_t* bytes);
+
+/* Zero the device status word (enqueued on stream). */
+tsa_status tsa_reset_device_status(void* ws, void* stream);
+
+/* Synchronise stream, read the device status word into *flags (may be NULL)
+ * and map it to a status: TSA_OK when no bit is set, else the first of
+ * TSA_ERR_TIMEOUT, TSA_ERR_BAD_INDEX, TSA_ERR_NONFINITE that is set. */
+tsa_status tsa_get_device_status(const void* ws, void* stream, uint32_t* flags);
+
+/* Step 1 -- proxy scores.  [GS] "Cobertura Dinamica de Tokens", scoring:
+ * for every (b, h) and window row i in [L-w, L), the causal softmax over keys
+ * j <= i of scale * q[b,h,i].k[b,h/G,j]; scores[b,h,j] is the sum of those
+ * weights over the w rows (fp32, accumulated in fp32/fp64).
+ * In: q, k.  Out: scores.  ws: >= tsa_stage_workspace_size bytes. */
+tsa_status tsa_score(const tsa_params* p, const void* q, const void* k, float* scores,
+                     void* ws, size_t ws_bytes, void* stream);
+
+/* Step 2 -- coverage budget.  [GS] "Cobertura Dinamica de Tokens", budget
+ * allocation and per-head selection: per head, masses
+ * q_j = ceil(score_j * 2^40) (int64), T = floor(tau * sum_j q_j) (fp64),
+ * p_h = the largest count of least-important tokens whose mass sum is <= T,
+ * k_head = L - p_h; the sequence's global budget k_seq[b] = max_h k_head.
+ * Bit-exact integer arithmetic.  Non-finite scores set TSA_DEVFLAG_NONFINITE.
+ * In: scores.  Out: k_head (may be NULL), k_seq.  ws: stage size. */
+tsa_status tsa_budget(const tsa_params* p, const float* scores, int32_t* k_head, int32_t* k_seq,
+                      void* ws, size_t ws_bytes, void* stream);
+
+/* Step 3 -- per-head top-k.  [GS] "Cobertura Dinamica de Tokens", per-head
+ * selection: S_h = the k_seq[b] tokens of largest score, equal scores going
+ * to the smaller index, written ascending to idx[b,h,0..k_b); the rest of
+ * idx[b,h,:] is set to -1.  In: scores, k_seq.  Out: idx.  ws: stage size. */
+tsa_status tsa_select(const tsa_params* p, const float* scores, const int32_t* k_seq, int32_t* idx,
+                      void* ws, size_t ws_bytes, void* stream);
+
+/* Step 4 -- gather.  [GS] "Arquitectura Central", compression:
+ * qc[b,h,i] = q[b,h,S_h[i]], kc[b,h,i] = k[b,h/G,S_h[i]],
+ * vc[b,h,i] = v[b,h/G,S_h[i]] for i < k_b.  Rows >= k_b are not written.
+ * An index outside [0, L) writes a zero row and sets TSA_DEVFLAG_BAD_INDEX
+ * (when ws is not NULL).  ws: NULL or stage size. */
+tsa_status tsa_gather_qkv(const tsa_params* p, const void* q, const void* k, const void* v,
+                          const int32_t* idx, const int32_t* k_seq, void* qc, void* kc, void* vc,
+                          void* ws, size_t ws_bytes, void* stream);
+
+/* Step 5 -- causal attention on the compressed tensors.  [GS] "Arquitectura
+ * Central": the compressed tensors stay dense, so an ordinary dense causal
+ * kernel runs on them.  oc[b,h,i] = sum_{j<=i} softmax_j(scale *
+ * qc[b,h,i].kc[b,h,j]) vc[b,h,j] for i < k_seq[b] (bf16 out, fp32
+ * accumulation; tcgen05 tensor cores).  Rows >= k_b of oc are not written.
+ * Rows of qc/kc/vc at or beyond k_b may hold any bits.  lse may be NULL.
+ * ws: stage size (its status word receives timeouts). */
+tsa_status tsa_attend(const tsa_params* p, const void* qc, const void* kc, const void* vc,
+                      const int32_t* k_seq, void* oc, float* lse,
+                      void* ws, size_t ws_bytes, void* stream);
+
+/* Dense causal GQA attention on the uncompressed tensors (the baseline the
+ * method is measured against; the same kernel as tsa_attend with the
+ * identity selection): o[b,h,i] = sum_{j<=i} softmax_j(scale *
+ * q[b,h,i].k[b,h/G,j]) v[b,h/G,j].  lse may be NULL.  ws: stage size. */
+tsa_status tsa_attend_dense(const tsa_params* p, const void* q, const void* k, const void* v,
+                            void* o, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/* Step 6 -- scatter.  [GS] "Arquitectura Central", decompression: o[b,h,:]
+ * is zero except o[b,h,S_h[i]] = oc[b,h,i] for i < k_b.  Every row of o is
+ * written exactly once.  ws: NULL or stage size. */
+tsa_status tsa_scatter(const tsa_params* p, const void* oc, const int32_t* idx, const int32_t* k_seq,
+                       void* o, void* ws, size_t ws_bytes, void* stream);
+
+/* The whole path: score -> budget -> select -> gather -> attend -> scatter,
+ * enqueued on stream with no host synchronisation.  scores_out, idx_out,
+ * k_seq_out may be NULL (then the workspace holds them); when given they
+ * receive the intermediate results.  ws: >= tsa_workspace_size bytes. */
+tsa_status tsa_forward(const tsa_params* p, const void* q, const void* k, const void* v, void* o,
+                       float* scores_out, int32_t* idx_out, int32_t* k_seq_out,
+                       void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TSA_H_ */

@@ -1,0 +1,254 @@
+"""Token Sparse Attention prefill path on NVIDIA B200 (sm_100a).
+
+Thin Python binding over the C ABI in ``include/tsa.h`` (``libtsa.so`` beside
+this file).  The functions here only marshal torch tensors into pointers and
+the current CUDA stream; every step of the path runs in the library's CUDA
+kernels.  There is no CPU fallback: if the library is missing or the tensors
+are not on a CUDA device, the calls raise.
+
+Names follow the C ABI: ``tsa_score``, ``tsa_budget``, ``tsa_select``,
+``tsa_gather_qkv``, ``tsa_attend``, ``tsa_attend_dense``, ``tsa_scatter``,
+``tsa_forward``, plus workspace and status helpers.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtsa.so")
+
+TSA_OK = 0
+STATUS_NAMES = {0: "TSA_OK", 1: "TSA_ERR_INVALID_ARG", 2: "TSA_ERR_UNSUPPORTED", 3: "TSA_ERR_WORKSPACE",
+                4: "TSA_ERR_CUDA", 5: "TSA_ERR_NONFINITE", 6: "TSA_ERR_TIMEOUT", 7: "TSA_ERR_BAD_INDEX"}
+DEVFLAG_NONFINITE, DEVFLAG_TIMEOUT, DEVFLAG_BAD_INDEX = 0x1, 0x2, 0x4
+
+# Every symbol the header declares (checked by the tests).
+EXPORTED = ("tsa_abi_version", "tsa_status_string", "tsa_check_params", "tsa_workspace_size",
+            "tsa_stage_workspace_size", "tsa_reset_device_status", "tsa_get_device_status",
+            "tsa_score", "tsa_budget", "tsa_select", "tsa_gather_qkv", "tsa_attend",
+            "tsa_attend_dense", "tsa_scatter", "tsa_forward")
+
+
+class TSAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)} ({_string(status)})")
+
+
+class tsa_params(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
+                ("L", ctypes.c_int32), ("d", ctypes.c_int32), ("w", ctypes.c_int32),
+                ("tau", ctypes.c_float), ("softmax_scale", ctypes.c_float),
+                ("flags", ctypes.c_uint32), ("timeout_ms", ctypes.c_uint32)]
+
+
+def params(B, Hq, Hkv, L, d, w, tau, softmax_scale=0.0, timeout_ms=0) -> tsa_params:
+    return tsa_params(B, Hq, Hkv, L, d, w, tau, softmax_scale, 0, timeout_ms)
+
+
+_lock = threading.Lock()
+_lib = None
+
+_P = ctypes.POINTER(tsa_params)
+_v = ctypes.c_void_p
+_sz = ctypes.c_size_t
+
+
+def load(path: str | None = None):
+    """Load ``libtsa.so`` (raises if it is absent: there is no fallback)."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        p = path or LIB_PATH
+        if not os.path.exists(p):
+            raise FileNotFoundError(f"{p} is missing; build it with token_sparse_attention_tsa_b200/build.py")
+        lib = ctypes.CDLL(p)
+        sig = {
+            "tsa_abi_version": ([], ctypes.c_int32),
+            "tsa_status_string": ([ctypes.c_int], ctypes.c_char_p),
+            "tsa_check_params": ([_P], ctypes.c_int),
+            "tsa_workspace_size": ([_P, ctypes.POINTER(_sz)], ctypes.c_int),
+            "tsa_stage_workspace_size": ([_P, ctypes.POINTER(_sz)], ctypes.c_int),
+            "tsa_reset_device_status": ([_v, _v], ctypes.c_int),
+            "tsa_get_device_status": ([_v, _v, ctypes.POINTER(ctypes.c_uint32)], ctypes.c_int),
+            "tsa_score": ([_P, _v, _v, _v, _v, _sz, _v], ctypes.c_int),
+            "tsa_budget": ([_P, _v, _v, _v, _v, _sz, _v], ctypes.c_int),
+            "tsa_select": ([_P, _v, _v, _v, _v, _sz, _v], ctypes.c_int),
+            "tsa_gather_qkv": ([_P, _v, _v, _v, _v, _v, _v, _v, _v, _v, _sz, _v], ctypes.c_int),
+            "tsa_attend": ([_P, _v, _v, _v, _v, _v, _v, _v, _sz, _v], ctypes.c_int),
+            "tsa_attend_dense": ([_P, _v, _v, _v, _v, _v, _v, _sz, _v], ctypes.c_int),
+            "tsa_scatter": ([_P, _v, _v, _v, _v, _v, _sz, _v], ctypes.c_int),
+            "tsa_forward": ([_P, _v, _v, _v, _v, _v, _v, _v, _v, _sz, _v], ctypes.c_int),
+        }
+        for name, (args, res) in sig.items():
+            fn = getattr(lib, name)
+            fn.argtypes = args
+            fn.restype = res
+        _lib = lib
+        return lib
+
+
+def _string(status: int) -> str:
+    try:
+        return load().tsa_status_string(status).decode()
+    except Exception:  # pragma: no cover
+        return "?"
+
+
+def _check(status: int, where: str):
+    if status != TSA_OK:
+        raise TSAError(status, where)
+
+
+def _ptr(t, name: str, dtype=None):
+    """Device pointer of a contiguous CUDA tensor (None -> NULL)."""
+    if t is None:
+        return None
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor (there is no CPU path)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
+    return t.data_ptr()
+
+
+def _stream(stream):
+    import torch
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _nbytes(t) -> int:
+    return t.numel() * t.element_size()
+
+
+# ---------------------------------------------------------------- sizing
+def workspace_size(p: tsa_params) -> int:
+    n = _sz()
+    _check(load().tsa_workspace_size(ctypes.byref(p), ctypes.byref(n)), "tsa_workspace_size")
+    return n.value
+
+
+def stage_workspace_size(p: tsa_params) -> int:
+    n = _sz()
+    _check(load().tsa_stage_workspace_size(ctypes.byref(p), ctypes.byref(n)), "tsa_stage_workspace_size")
+    return n.value
+
+
+def check_params(p: tsa_params) -> int:
+    """Status code of the host-side validation (no exception)."""
+    return load().tsa_check_params(ctypes.byref(p))
+
+
+def new_workspace(p: tsa_params, full: bool = True, device=None):
+    """A uint8 CUDA tensor sized for tsa_forward (full) or the stage calls,
+    with its status word cleared."""
+    import torch
+    n = workspace_size(p) if full else stage_workspace_size(p)
+    ws = torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+    reset_device_status(ws)
+    return ws
+
+
+def reset_device_status(ws, stream=None):
+    _check(load().tsa_reset_device_status(_ptr(ws, "ws"), _stream(stream)), "tsa_reset_device_status")
+
+
+def get_device_status(ws, stream=None) -> tuple[int, int]:
+    """(status code, raw flag bits) of the device status word; synchronises."""
+    flags = ctypes.c_uint32()
+    st = load().tsa_get_device_status(_ptr(ws, "ws"), _stream(stream), ctypes.byref(flags))
+    return st, flags.value
+
+
+# ---------------------------------------------------------------- stages
+def tsa_score(p, q, k, scores, ws, stream=None):
+    import torch
+    _check(load().tsa_score(ctypes.byref(p), _ptr(q, "q", torch.bfloat16), _ptr(k, "k", torch.bfloat16),
+                            _ptr(scores, "scores", torch.float32), _ptr(ws, "ws"), _nbytes(ws),
+                            _stream(stream)), "tsa_score")
+
+
+def tsa_budget(p, scores, k_head, k_seq, ws, stream=None):
+    import torch
+    _check(load().tsa_budget(ctypes.byref(p), _ptr(scores, "scores", torch.float32),
+                             _ptr(k_head, "k_head", torch.int32), _ptr(k_seq, "k_seq", torch.int32),
+                             _ptr(ws, "ws"), _nbytes(ws), _stream(stream)), "tsa_budget")
+
+
+def tsa_select(p, scores, k_seq, idx, ws, stream=None):
+    import torch
+    _check(load().tsa_select(ctypes.byref(p), _ptr(scores, "scores", torch.float32),
+                             _ptr(k_seq, "k_seq", torch.int32), _ptr(idx, "idx", torch.int32),
+                             _ptr(ws, "ws"), _nbytes(ws), _stream(stream)), "tsa_select")
+
+
+def tsa_gather_qkv(p, q, k, v, idx, k_seq, qc, kc, vc, ws=None, stream=None):
+    import torch
+    bf = torch.bfloat16
+    _check(load().tsa_gather_qkv(ctypes.byref(p), _ptr(q, "q", bf), _ptr(k, "k", bf), _ptr(v, "v", bf),
+                                 _ptr(idx, "idx", torch.int32), _ptr(k_seq, "k_seq", torch.int32),
+                                 _ptr(qc, "qc", bf), _ptr(kc, "kc", bf), _ptr(vc, "vc", bf),
+                                 _ptr(ws, "ws"), _nbytes(ws) if ws is not None else 0, _stream(stream)),
+           "tsa_gather_qkv")
+
+
+def tsa_attend(p, qc, kc, vc, k_seq, oc, lse, ws, stream=None):
+    import torch
+    bf = torch.bfloat16
+    _check(load().tsa_attend(ctypes.byref(p), _ptr(qc, "qc", bf), _ptr(kc, "kc", bf), _ptr(vc, "vc", bf),
+                             _ptr(k_seq, "k_seq", torch.int32), _ptr(oc, "oc", bf),
+                             _ptr(lse, "lse", torch.float32), _ptr(ws, "ws"), _nbytes(ws), _stream(stream)),
+           "tsa_attend")
+
+
+def tsa_attend_dense(p, q, k, v, o, lse, ws, stream=None):
+    import torch
+    bf = torch.bfloat16
+    _check(load().tsa_attend_dense(ctypes.byref(p), _ptr(q, "q", bf), _ptr(k, "k", bf), _ptr(v, "v", bf),
+                                   _ptr(o, "o", bf), _ptr(lse, "lse", torch.float32), _ptr(ws, "ws"),
+                                   _nbytes(ws), _stream(stream)), "tsa_attend_dense")
+
+
+def tsa_scatter(p, oc, idx, k_seq, o, ws=None, stream=None):
+    import torch
+    bf = torch.bfloat16
+    _check(load().tsa_scatter(ctypes.byref(p), _ptr(oc, "oc", bf), _ptr(idx, "idx", torch.int32),
+                              _ptr(k_seq, "k_seq", torch.int32), _ptr(o, "o", bf), _ptr(ws, "ws"),
+                              _nbytes(ws) if ws is not None else 0, _stream(stream)), "tsa_scatter")
+
+
+def tsa_forward(p, q, k, v, o, ws, scores_out=None, idx_out=None, k_seq_out=None, stream=None):
+    import torch
+    bf = torch.bfloat16
+    _check(load().tsa_forward(ctypes.byref(p), _ptr(q, "q", bf), _ptr(k, "k", bf), _ptr(v, "v", bf),
+                              _ptr(o, "o", bf), _ptr(scores_out, "scores_out", torch.float32),
+                              _ptr(idx_out, "idx_out", torch.int32), _ptr(k_seq_out, "k_seq_out", torch.int32),
+                              _ptr(ws, "ws"), _nbytes(ws), _stream(stream)), "tsa_forward")
+
+
+def forward(q, k, v, w: int, tau: float, softmax_scale: float = 0.0, ws=None, return_intermediates=False):
+    """Convenience wrapper: allocate the output (and workspace if not given)
+    and run ``tsa_forward`` on the current stream."""
+    import torch
+    B, Hq, L, d = q.shape
+    Hkv = k.shape[1]
+    p = params(B, Hq, Hkv, L, d, w, tau, softmax_scale)
+    if ws is None:
+        ws = new_workspace(p, full=True, device=q.device)
+    o = torch.empty_like(q)
+    if not return_intermediates:
+        tsa_forward(p, q, k, v, o, ws)
+        return o
+    scores = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device)
+    idx = torch.empty((B, Hq, L), dtype=torch.int32, device=q.device)
+    k_seq = torch.empty((B,), dtype=torch.int32, device=q.device)
+    tsa_forward(p, q, k, v, o, ws, scores, idx, k_seq)
+    return o, scores, idx, k_seq

@@ -1,0 +1,124 @@
+// copy.cuh -- gather of Q/K/V into compressed tensors and scatter of the
+// compressed output back to full length.
+//
+// Source: gist.science summary page "Token Sparse Attention: Efficient
+// Long-Context Inference with Interleaved Token Selection", section 2,
+// "Arquitectura Central": compression gathers each head's selected rows of
+// Q, K and V into dense, contiguous tensors; decompression places each row of
+// the compressed output back at its token position in an output that is zero
+// everywhere else.
+//
+// Both kernels are pure HBM traffic: each row (d bf16 = 128 or 256 bytes) is
+// moved by d/8 lanes with one 16-byte load and store per lane, so a warp moves
+// whole rows with full 32-byte sectors.
+#pragma once
+
+#include <cuda_bf16.h>
+
+namespace tsa {
+
+struct GatherArgs {
+  const __nv_bfloat16 *q, *k, *v;  // [B*Hq, L, D], [B*Hkv, L, D] x2
+  const int32_t* idx;              // [B*Hq, L]
+  const int32_t* k_seq;            // [B]
+  __nv_bfloat16 *qc, *kc, *vc;     // [B*Hq, L, D]
+  uint32_t* status;                // or null
+  int L, Hq, Hkv, G;
+  long long total_rows;            // B*Hq*L
+};
+
+template <int D>
+__global__ void __launch_bounds__(256) gather_kernel(const GatherArgs a) {
+  constexpr int LPR = D / 8;  // lanes per row
+  const int sub = threadIdx.x % LPR;
+  const long long stride = static_cast<long long>(gridDim.x) * (blockDim.x / LPR);
+  bool bad = false;
+  for (long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) / LPR;
+       row < a.total_rows; row += stride) {
+    const long long bh = row / a.L;
+    const int i = static_cast<int>(row - bh * a.L);
+    const int b = static_cast<int>(bh / a.Hq);
+    const int h = static_cast<int>(bh - static_cast<long long>(b) * a.Hq);
+    const int kb = __ldg(a.k_seq + b);
+    if (i >= kb) continue;
+    const int j = __ldg(a.idx + row);
+    const size_t dst = static_cast<size_t>(row) * D + sub * 8;
+    if (j < 0 || j >= a.L) {
+      bad = true;
+      const uint4 z = make_uint4(0, 0, 0, 0);
+      *reinterpret_cast<uint4*>(a.qc + dst) = z;
+      *reinterpret_cast<uint4*>(a.kc + dst) = z;
+      *reinterpret_cast<uint4*>(a.vc + dst) = z;
+      continue;
+    }
+    const size_t sq = (static_cast<size_t>(bh) * a.L + j) * D + sub * 8;
+    const size_t skv = ((static_cast<size_t>(b) * a.Hkv + h / a.G) * a.L + j) * D + sub * 8;
+    const uint4 vq = __ldg(reinterpret_cast<const uint4*>(a.q + sq));
+    const uint4 vk = __ldg(reinterpret_cast<const uint4*>(a.k + skv));
+    const uint4 vv = __ldg(reinterpret_cast<const uint4*>(a.v + skv));
+    *reinterpret_cast<uint4*>(a.qc + dst) = vq;
+    *reinterpret_cast<uint4*>(a.kc + dst) = vk;
+    *reinterpret_cast<uint4*>(a.vc + dst) = vv;
+  }
+  if (bad && a.status) atomicOr(a.status, 0x4u);
+}
+
+struct ScatterArgs {
+  const __nv_bfloat16* oc;  // [B*Hq, L, D]
+  const int32_t* idx;       // [B*Hq, L]
+  const int32_t* k_seq;     // [B]
+  __nv_bfloat16* o;         // [B*Hq, L, D]
+  uint32_t* status;         // or null
+  int L, Hq;
+};
+
+constexpr int SCAT_ROWS = 256;  // output rows per CTA
+
+// grid (ceil(L/256), B*Hq), 256 threads.  The CTA maps its 256 output rows to
+// compressed positions through a shared table built from the ascending idx
+// (one binary search for the first entry), then writes every row once.
+template <int D>
+__global__ void __launch_bounds__(256) scatter_kernel(const ScatterArgs a) {
+  constexpr int LPR = D / 8;
+  __shared__ int32_t where[SCAT_ROWS];
+  __shared__ int32_t s_first;
+  const int bh = blockIdx.y;
+  const int r0 = blockIdx.x * SCAT_ROWS;
+  const int b = bh / a.Hq;
+  int kb = __ldg(a.k_seq + b);
+  kb = kb < 0 ? 0 : (kb > a.L ? a.L : kb);
+  const int32_t* ix = a.idx + static_cast<size_t>(bh) * a.L;
+  where[threadIdx.x] = -1;
+  if (threadIdx.x == 0) {  // first i with ix[i] >= r0
+    int lo = 0, hi = kb;
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if (__ldg(ix + mid) < r0) lo = mid + 1; else hi = mid;
+    }
+    s_first = lo;
+  }
+  __syncthreads();
+  bool bad = false;
+  {
+    const int i = s_first + threadIdx.x;
+    if (i < kb) {
+      const int r = __ldg(ix + i) - r0;
+      if (r >= 0 && r < SCAT_ROWS) where[r] = i;
+      else if (r + r0 < 0 || r + r0 >= a.L) bad = true;
+    }
+  }
+  __syncthreads();
+  const int sub = threadIdx.x % LPR;
+  constexpr int ROWS_PER_PASS = 256 / LPR;
+  for (int rr = threadIdx.x / LPR; rr < SCAT_ROWS; rr += ROWS_PER_PASS) {
+    const int r = r0 + rr;
+    if (r >= a.L) break;
+    const int i = where[rr];
+    uint4 val = make_uint4(0, 0, 0, 0);
+    if (i >= 0) val = __ldg(reinterpret_cast<const uint4*>(a.oc + (static_cast<size_t>(bh) * a.L + i) * D + sub * 8));
+    __stcs(reinterpret_cast<uint4*>(a.o + (static_cast<size_t>(bh) * a.L + r) * D + sub * 8), val);
+  }
+  if (bad && a.status) atomicOr(a.status, 0x4u);
+}
+
+}  // namespace tsa

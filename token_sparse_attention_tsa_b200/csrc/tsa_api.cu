@@ -1,0 +1,456 @@
+// tsa_api.cu -- host side of the C ABI declared in include/tsa.h: argument
+// validation, workspace carving, TMA descriptor encoding and kernel launches
+// for the Token Sparse Attention prefill path on sm_100a.
+//
+// Method source: gist.science summary page "Token Sparse Attention: Efficient
+// Long-Context Inference with Interleaved Token Selection", section 2
+// ("Arquitectura Central", "Cobertura Dinamica de Tokens"); each kernel file
+// cites the part it implements.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "tsa.h"
+#include "attend.cuh"
+#include "copy.cuh"
+#include "score.cuh"
+#include "select.cuh"
+
+namespace {
+
+using tsa::AttnLayout;
+
+constexpr size_t kAlign = 256;
+constexpr int kMaxDevices = 64;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int score_chunks(const tsa_params* p) {
+  const int span = tsa::SC_CHUNK_TILES * tsa::SC_KEYS;
+  return (p->L + span - 1) / span;
+}
+
+// Workspace layout.  Stage part: status word (+ abort word), score scratch.
+// Forward part: scores, idx, k_head, k_seq, qc, kc, vc, oc.
+struct WsLayout {
+  size_t status = 0, part_m = 0, part_z = 0, stats = 0, stage_end = 0;
+  size_t scores = 0, idx = 0, k_head = 0, k_seq = 0, qc = 0, kc = 0, vc = 0, oc = 0, total = 0;
+};
+
+WsLayout layout_of(const tsa_params* p) {
+  WsLayout w;
+  const size_t bhq = static_cast<size_t>(p->B) * p->Hq;
+  const size_t rows = bhq * static_cast<size_t>(p->w);
+  const size_t nch = static_cast<size_t>(score_chunks(p));
+  size_t off = 0;
+  w.status = off;           off += kAlign;
+  w.part_m = off;           off = align_up(off + rows * nch * sizeof(float));
+  w.part_z = off;           off = align_up(off + rows * nch * sizeof(double));
+  w.stats = off;            off = align_up(off + rows * sizeof(float2));
+  w.stage_end = off;
+  const size_t tok = bhq * static_cast<size_t>(p->L);
+  const size_t ten = tok * static_cast<size_t>(p->d) * 2;
+  w.scores = off;           off = align_up(off + tok * sizeof(float));
+  w.idx = off;              off = align_up(off + tok * sizeof(int32_t));
+  w.k_head = off;           off = align_up(off + bhq * sizeof(int32_t));
+  w.k_seq = off;            off = align_up(off + static_cast<size_t>(p->B) * sizeof(int32_t));
+  w.qc = off;               off = align_up(off + ten);
+  w.kc = off;               off = align_up(off + ten);
+  w.vc = off;               off = align_up(off + ten);
+  w.oc = off;               off = align_up(off + ten);
+  w.total = off;
+  return w;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+float scale_of(const tsa_params* p) {
+  return p->softmax_scale > 0.f ? p->softmax_scale : 1.0f / std::sqrt(static_cast<float>(p->d));
+}
+
+uint64_t limit_ns_of(const tsa_params* p) {
+  const uint64_t ms = p->timeout_ms ? p->timeout_ms : 2000u;
+  return ms * 1000000ull;
+}
+
+tsa_status cuda_ok(cudaError_t e) { return e == cudaSuccess ? TSA_OK : TSA_ERR_CUDA; }
+
+tsa_status launch_ok() { return cuda_ok(cudaGetLastError()); }
+
+// ---------------------------------------------------------------- TMA maps
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// [heads, L, d] bf16 rows; box = 128 rows x 64 columns, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, int d, int L, int heads) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(heads)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(L) * d * 2};
+  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------- attributes
+template <typename K>
+bool ensure_smem(std::atomic<int> (&done)[kMaxDevices], K kernel, int bytes) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  if (done[dev].load(std::memory_order_acquire)) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess)
+    return false;
+  done[dev].store(1, std::memory_order_release);
+  return true;
+}
+
+std::atomic<int> g_attn64[kMaxDevices], g_attn128[kMaxDevices], g_st64[kMaxDevices],
+    g_st128[kMaxDevices], g_sum64[kMaxDevices], g_sum128[kMaxDevices], g_budget[kMaxDevices],
+    g_select[kMaxDevices];
+
+constexpr int kBudgetSmem = tsa::BS_WARPS * 256 * (8 + 4);
+constexpr int kSelectSmem = tsa::BS_WARPS * 256 * 4;
+
+// ---------------------------------------------------------------- launchers
+tsa_status run_score(const tsa_params* p, const void* q, const void* k, float* scores, void* ws,
+                     cudaStream_t st) {
+  const WsLayout w = layout_of(p);
+  tsa::ScoreArgs a;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.k = static_cast<const __nv_bfloat16*>(k);
+  a.scores = scores;
+  a.part_m = at<float>(ws, w.part_m);
+  a.part_z = at<double>(ws, w.part_z);
+  a.stats = at<float2>(ws, w.stats);
+  a.L = p->L;
+  a.w = p->w;
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.G = p->Hq / p->Hkv;
+  a.n_chunks = score_chunks(p);
+  a.scale = scale_of(p);
+  const int bhq = p->B * p->Hq;
+  const dim3 g1(a.n_chunks, bhq), g2((p->L + tsa::SC_KEYS - 1) / tsa::SC_KEYS, bhq);
+  const int sm1 = 2 * p->d * 128 * 4;
+  const int sm2 = sm1 + 16 * 128 * 4;
+  const int rows = bhq * p->w;
+  if (p->d == 128) {
+    if (!ensure_smem(g_st128, tsa::score_stats_kernel<128>, sm1) ||
+        !ensure_smem(g_sum128, tsa::score_sum_kernel<128>, sm2))
+      return TSA_ERR_CUDA;
+    tsa::score_stats_kernel<128><<<g1, tsa::SC_THREADS, sm1, st>>>(a);
+    tsa::score_merge_kernel<<<(rows + 255) / 256, 256, 0, st>>>(a, rows);
+    tsa::score_sum_kernel<128><<<g2, tsa::SC_THREADS, sm2, st>>>(a);
+  } else {
+    if (!ensure_smem(g_st64, tsa::score_stats_kernel<64>, sm1) ||
+        !ensure_smem(g_sum64, tsa::score_sum_kernel<64>, sm2))
+      return TSA_ERR_CUDA;
+    tsa::score_stats_kernel<64><<<g1, tsa::SC_THREADS, sm1, st>>>(a);
+    tsa::score_merge_kernel<<<(rows + 255) / 256, 256, 0, st>>>(a, rows);
+    tsa::score_sum_kernel<64><<<g2, tsa::SC_THREADS, sm2, st>>>(a);
+  }
+  return launch_ok();
+}
+
+tsa_status run_budget(const tsa_params* p, const float* scores, int32_t* k_head, int32_t* k_seq,
+                      uint32_t* status, cudaStream_t st) {
+  if (!ensure_smem(g_budget, tsa::budget_kernel, kBudgetSmem)) return TSA_ERR_CUDA;
+  if (cudaMemsetAsync(k_seq, 0, sizeof(int32_t) * p->B, st) != cudaSuccess) return TSA_ERR_CUDA;
+  tsa::BudgetArgs a{scores, k_head, k_seq, status, p->L, p->Hq,
+                    static_cast<double>(p->tau)};
+  tsa::budget_kernel<<<p->B * p->Hq, tsa::BS_THREADS, kBudgetSmem, st>>>(a);
+  return launch_ok();
+}
+
+tsa_status run_select(const tsa_params* p, const float* scores, const int32_t* k_seq, int32_t* idx,
+                      cudaStream_t st) {
+  if (!ensure_smem(g_select, tsa::select_kernel, kSelectSmem)) return TSA_ERR_CUDA;
+  tsa::SelectArgs a{scores, k_seq, idx, p->L, p->Hq};
+  tsa::select_kernel<<<p->B * p->Hq, tsa::BS_THREADS, kSelectSmem, st>>>(a);
+  return launch_ok();
+}
+
+int copy_grid(long long rows, int lanes_per_row) {
+  long long blocks = (rows * lanes_per_row + 255) / 256;
+  const long long cap = 148LL * 8;
+  return static_cast<int>(blocks < cap ? (blocks < 1 ? 1 : blocks) : cap);
+}
+
+tsa_status run_gather(const tsa_params* p, const void* q, const void* k, const void* v, const int32_t* idx,
+                      const int32_t* k_seq, void* qc, void* kc, void* vc, uint32_t* status, cudaStream_t st) {
+  tsa::GatherArgs a;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.k = static_cast<const __nv_bfloat16*>(k);
+  a.v = static_cast<const __nv_bfloat16*>(v);
+  a.idx = idx;
+  a.k_seq = k_seq;
+  a.qc = static_cast<__nv_bfloat16*>(qc);
+  a.kc = static_cast<__nv_bfloat16*>(kc);
+  a.vc = static_cast<__nv_bfloat16*>(vc);
+  a.status = status;
+  a.L = p->L;
+  a.Hq = p->Hq;
+  a.Hkv = p->Hkv;
+  a.G = p->Hq / p->Hkv;
+  a.total_rows = static_cast<long long>(p->B) * p->Hq * p->L;
+  if (p->d == 128)
+    tsa::gather_kernel<128><<<copy_grid(a.total_rows, 16), 256, 0, st>>>(a);
+  else
+    tsa::gather_kernel<64><<<copy_grid(a.total_rows, 8), 256, 0, st>>>(a);
+  return launch_ok();
+}
+
+tsa_status run_scatter(const tsa_params* p, const void* oc, const int32_t* idx, const int32_t* k_seq, void* o,
+                       uint32_t* status, cudaStream_t st) {
+  tsa::ScatterArgs a{static_cast<const __nv_bfloat16*>(oc), idx, k_seq, static_cast<__nv_bfloat16*>(o),
+                     status, p->L, p->Hq};
+  const dim3 g((p->L + tsa::SCAT_ROWS - 1) / tsa::SCAT_ROWS, p->B * p->Hq);
+  if (p->d == 128)
+    tsa::scatter_kernel<128><<<g, 256, 0, st>>>(a);
+  else
+    tsa::scatter_kernel<64><<<g, 256, 0, st>>>(a);
+  return launch_ok();
+}
+
+// Attention over [B*Hq, L, d] queries against K/V with heads_kv heads
+// (query head h of sequence b reads K/V head b*heads_kv + h/g_kv).
+tsa_status run_attend(const tsa_params* p, const void* q, const void* k, const void* v, int heads_kv, int g_kv,
+                      const int32_t* k_seq, void* o, float* lse, uint32_t* status, uint32_t* abort_word,
+                      cudaStream_t st) {
+  CUtensorMap mq, mk, mv;
+  const int bhq = p->B * p->Hq;
+  const int bhkv = p->B * heads_kv;
+  if (!make_map(&mq, q, p->d, p->L, bhq) || !make_map(&mk, k, p->d, p->L, bhkv) ||
+      !make_map(&mv, v, p->d, p->L, bhkv))
+    return TSA_ERR_CUDA;
+  if (cudaMemsetAsync(abort_word, 0, sizeof(uint32_t), st) != cudaSuccess) return TSA_ERR_CUDA;
+  tsa::AttnArgs a;
+  a.k_seq = k_seq;
+  a.o = static_cast<__nv_bfloat16*>(o);
+  a.lse = lse;
+  a.status = status;
+  a.abort_word = abort_word;
+  a.L = p->L;
+  a.Hq = p->Hq;
+  a.Hkv_map = heads_kv;
+  a.G_map = g_kv;
+  a.n_tiles = (p->L + 127) / 128;
+  a.scale_log2 = scale_of(p) * 1.4426950408889634f;
+  a.limit_ns = limit_ns_of(p);
+  const dim3 grid(a.n_tiles, bhq);
+  if (p->d == 128) {
+    constexpr int sm = AttnLayout<128>::ALLOC;
+    if (!ensure_smem(g_attn128, tsa::attend_kernel<128>, sm)) return TSA_ERR_CUDA;
+    tsa::attend_kernel<128><<<grid, 192, sm, st>>>(mq, mk, mv, a);
+  } else {
+    constexpr int sm = AttnLayout<64>::ALLOC;
+    if (!ensure_smem(g_attn64, tsa::attend_kernel<64>, sm)) return TSA_ERR_CUDA;
+    tsa::attend_kernel<64><<<grid, 192, sm, st>>>(mq, mk, mv, a);
+  }
+  return launch_ok();
+}
+
+tsa_status check_ws(const tsa_params* p, void* ws, size_t ws_bytes, bool full) {
+  if (!ws) return TSA_ERR_WORKSPACE;
+  if (!aligned(ws, kAlign)) return TSA_ERR_INVALID_ARG;
+  const WsLayout w = layout_of(p);
+  if (ws_bytes < (full ? w.total : w.stage_end)) return TSA_ERR_WORKSPACE;
+  return TSA_OK;
+}
+
+bool tensors_ok(std::initializer_list<const void*> ptrs) {
+  for (const void* q : ptrs)
+    if (!q || !aligned(q, 16)) return false;
+  return true;
+}
+
+uint32_t* status_of(void* ws) { return ws ? at<uint32_t>(ws, 0) : nullptr; }
+uint32_t* abort_of(void* ws) { return at<uint32_t>(ws, 4); }
+
+}  // namespace
+
+extern "C" {
+
+int32_t tsa_abi_version(void) { return TSA_ABI_VERSION; }
+
+const char* tsa_status_string(tsa_status s) {
+  switch (s) {
+    case TSA_OK: return "ok";
+    case TSA_ERR_INVALID_ARG: return "invalid argument";
+    case TSA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case TSA_ERR_WORKSPACE: return "workspace missing or too small";
+    case TSA_ERR_CUDA: return "CUDA error";
+    case TSA_ERR_NONFINITE: return "non-finite or negative score";
+    case TSA_ERR_TIMEOUT: return "pipeline wait timed out";
+    case TSA_ERR_BAD_INDEX: return "index outside [0, L)";
+  }
+  return "unknown status";
+}
+
+tsa_status tsa_check_params(const tsa_params* p) {
+  if (!p) return TSA_ERR_INVALID_ARG;
+  if (p->B < 1 || p->Hq < 1 || p->Hkv < 1 || p->L < 1 || p->d < 1 || p->w < 1) return TSA_ERR_INVALID_ARG;
+  if (p->Hq % p->Hkv != 0) return TSA_ERR_INVALID_ARG;
+  if (p->w > p->L) return TSA_ERR_INVALID_ARG;
+  if (!(p->tau >= 0.f && p->tau < 1.f)) return TSA_ERR_INVALID_ARG;
+  if (!(p->softmax_scale >= 0.f) || std::isinf(p->softmax_scale)) return TSA_ERR_INVALID_ARG;
+  if (p->flags != 0) return TSA_ERR_INVALID_ARG;
+  if (p->d != 64 && p->d != 128) return TSA_ERR_UNSUPPORTED;
+  if (p->w > 4096 || p->L > (1 << 22)) return TSA_ERR_UNSUPPORTED;
+  if (static_cast<long long>(p->B) * p->Hq * p->L >= (1LL << 31)) return TSA_ERR_UNSUPPORTED;
+  return TSA_OK;
+}
+
+tsa_status tsa_workspace_size(const tsa_params* p, size_t* bytes) {
+  const tsa_status s = tsa_check_params(p);
+  if (s != TSA_OK) return s;
+  if (!bytes) return TSA_ERR_INVALID_ARG;
+  *bytes = layout_of(p).total;
+  return TSA_OK;
+}
+
+tsa_status tsa_stage_workspace_size(const tsa_params* p, size_t* bytes) {
+  const tsa_status s = tsa_check_params(p);
+  if (s != TSA_OK) return s;
+  if (!bytes) return TSA_ERR_INVALID_ARG;
+  *bytes = layout_of(p).stage_end;
+  return TSA_OK;
+}
+
+tsa_status tsa_reset_device_status(void* ws, void* stream) {
+  if (!ws || !aligned(ws, kAlign)) return TSA_ERR_INVALID_ARG;
+  return cuda_ok(cudaMemsetAsync(ws, 0, 8, static_cast<cudaStream_t>(stream)));
+}
+
+tsa_status tsa_get_device_status(const void* ws, void* stream, uint32_t* flags) {
+  if (!ws || !aligned(ws, kAlign)) return TSA_ERR_INVALID_ARG;
+  uint32_t v = 0;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(&v, ws, sizeof(v), cudaMemcpyDeviceToHost, st) != cudaSuccess) return TSA_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return TSA_ERR_CUDA;
+  if (flags) *flags = v;
+  if (v & TSA_DEVFLAG_TIMEOUT) return TSA_ERR_TIMEOUT;
+  if (v & TSA_DEVFLAG_BAD_INDEX) return TSA_ERR_BAD_INDEX;
+  if (v & TSA_DEVFLAG_NONFINITE) return TSA_ERR_NONFINITE;
+  return TSA_OK;
+}
+
+tsa_status tsa_score(const tsa_params* p, const void* q, const void* k, float* scores, void* ws,
+                     size_t ws_bytes, void* stream) {
+  tsa_status s = tsa_check_params(p);
+  if (s != TSA_OK) return s;
+  if (!tensors_ok({q, k, scores})) return TSA_ERR_INVALID_ARG;
+  if ((s = check_ws(p, ws, ws_bytes, false)) != TSA_OK) return s;
+  return run_score(p, q, k, scores, ws, static_cast<cudaStream_t>(stream));
+}
+
+tsa_status tsa_budget(const tsa_params* p, const float* scores, int32_t* k_head, int32_t* k_seq, void* ws,
+                      size_t ws_bytes, void* stream) {
+  tsa_status s = tsa_check_params(p);
+  if (s != TSA_OK) return s;
+  if (!tensors_ok({scores, k_seq}) || (k_head && !aligned(k_head, 4))) return TSA_ERR_INVALID_ARG;
+  if ((s = check_ws(p, ws, ws_bytes, false)) != TSA_OK) return s;
+  return run_budget(p, scores, k_head, k_seq, status_of(ws), static_cast<cudaStream_t>(stream));
+}
+
+tsa_status tsa_select(const tsa_params* p, const float* scores, const int32_t* k_seq, int32_t* idx, void* ws,
+                      size_t ws_bytes, void* stream) {
+  tsa_status s = tsa_check_params(p);
+  if (s != TSA_OK) return s;
+  if (!tensors_ok({scores, k_seq, idx})) return TSA_ERR_INVALID_ARG;
+  if ((s = check_ws(p, ws, ws_bytes, false)) != TSA_OK) return s;
+  return run_select(p, scores, k_seq, idx, static_cast<cudaStream_t>(stream));
+}
+
+tsa_status tsa_gather_qkv(const tsa_params* p, const void* q, const void* k, const void* v, const int32_t* idx,
+                          const int32_t* k_seq, void* qc, void* kc, void* vc, void* ws, size_t ws_bytes,
+                          void* stream) {
+  tsa_status s = tsa_check_params(p);
+  if (s != TSA_OK) return s;
+  if (!tensors_ok({q, k, v, idx, k_seq, qc, kc, vc})) return TSA_ERR_INVALID_ARG;
+  if (ws && (s = check_ws(p, ws, ws_bytes, false)) != TSA_OK) return s;
+  return run_gather(p, q, k, v, idx, k_seq, qc, kc, vc, status_of(ws), static_cast<cudaStream_t>(stream));
+}
+
+tsa_status tsa_attend(const tsa_params* p, const void* qc, const void* kc, const void* vc, const int32_t* k_seq,
+                      void* oc, float* lse, void* ws, size_t ws_bytes, void* stream) {
+  tsa_status s = tsa_check_params(p);
+  if (s != TSA_OK) return s;
+  if (!tensors_ok({qc, kc, vc, k_seq, oc}) || (lse && !aligned(lse, 4))) return TSA_ERR_INVALID_ARG;
+  if ((s = check_ws(p, ws, ws_bytes, false)) != TSA_OK) return s;
+  return run_attend(p, qc, kc, vc, p->Hq, 1, k_seq, oc, lse, status_of(ws), abort_of(ws),
+                    static_cast<cudaStream_t>(stream));
+}
+
+tsa_status tsa_attend_dense(const tsa_params* p, const void* q, const void* k, const void* v, void* o,
+                            float* lse, void* ws, size_t ws_bytes, void* stream) {
+  tsa_status s = tsa_check_params(p);
+  if (s != TSA_OK) return s;
+  if (!tensors_ok({q, k, v, o}) || (lse && !aligned(lse, 4))) return TSA_ERR_INVALID_ARG;
+  if ((s = check_ws(p, ws, ws_bytes, false)) != TSA_OK) return s;
+  return run_attend(p, q, k, v, p->Hkv, p->Hq / p->Hkv, nullptr, o, lse, status_of(ws), abort_of(ws),
+                    static_cast<cudaStream_t>(stream));
+}
+
+tsa_status tsa_scatter(const tsa_params* p, const void* oc, const int32_t* idx, const int32_t* k_seq, void* o,
+                       void* ws, size_t ws_bytes, void* stream) {
+  tsa_status s = tsa_check_params(p);
+  if (s != TSA_OK) return s;
+  if (!tensors_ok({oc, idx, k_seq, o})) return TSA_ERR_INVALID_ARG;
+  if (ws && (s = check_ws(p, ws, ws_bytes, false)) != TSA_OK) return s;
+  return run_scatter(p, oc, idx, k_seq, o, status_of(ws), static_cast<cudaStream_t>(stream));
+}
+
+tsa_status tsa_forward(const tsa_params* p, const void* q, const void* k, const void* v, void* o,
+                       float* scores_out, int32_t* idx_out, int32_t* k_seq_out, void* ws, size_t ws_bytes,
+                       void* stream) {
+  tsa_status s = tsa_check_params(p);
+  if (s != TSA_OK) return s;
+  if (!tensors_ok({q, k, v, o})) return TSA_ERR_INVALID_ARG;
+  if ((scores_out && !aligned(scores_out, 16)) || (idx_out && !aligned(idx_out, 16)) ||
+      (k_seq_out && !aligned(k_seq_out, 4)))
+    return TSA_ERR_INVALID_ARG;
+  if ((s = check_ws(p, ws, ws_bytes, true)) != TSA_OK) return s;
+  const WsLayout w = layout_of(p);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* scores = scores_out ? scores_out : at<float>(ws, w.scores);
+  int32_t* idx = idx_out ? idx_out : at<int32_t>(ws, w.idx);
+  int32_t* kseq = k_seq_out ? k_seq_out : at<int32_t>(ws, w.k_seq);
+  void* qc = at<void>(ws, w.qc);
+  void* kc = at<void>(ws, w.kc);
+  void* vc = at<void>(ws, w.vc);
+  void* oc = at<void>(ws, w.oc);
+  if ((s = run_score(p, q, k, scores, ws, st)) != TSA_OK) return s;
+  if ((s = run_budget(p, scores, at<int32_t>(ws, w.k_head), kseq, status_of(ws), st)) != TSA_OK) return s;
+  if ((s = run_select(p, scores, kseq, idx, st)) != TSA_OK) return s;
+  if ((s = run_gather(p, q, k, v, idx, kseq, qc, kc, vc, status_of(ws), st)) != TSA_OK) return s;
+  if ((s = run_attend(p, qc, kc, vc, p->Hq, 1, kseq, oc, nullptr, status_of(ws), abort_of(ws), st)) != TSA_OK)
+    return s;
+  return run_scatter(p, oc, idx, kseq, o, status_of(ws), st);
+}
+
+}  // extern "C"
