@@ -57,6 +57,28 @@ def peaks() -> dict:
     return {"hbm_gbs": 6650.0, "bf16": 1590.0, "bf16_sustained": 1400.0, "source": "fallback"}
 
 
+# ---------------------------------------------------------------- ranks
+def rank_workload(wl, rank: int):
+    """Each rank processes its own sequence(s): same shape, own seed."""
+    return wl.with_(seed=wl.seed + 1000 * rank)
+
+
+def max_over_ranks(x: float, dist, device) -> float:
+    """Step time of the whole job: the slowest rank (identity without dist)."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_value(wl, world: int, ms: float) -> float:
+    """Whole-job effective TFLOP/s: every rank's dense-equivalent FLOPs over
+    the max-over-ranks step time."""
+    return world * dense_flops(wl) / (ms * 1e-3) / 1e12
+
+
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons during timing."""
@@ -194,15 +216,11 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
         if dist is not None:
             dist.barrier()
 
-    def max_over_ranks(x: float) -> float:
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def rank_max(x: float) -> float:
+        return max_over_ranks(x, dist, dev)
 
-    # inputs: this rank's own sequence (seed offset by rank)
-    wl_r = wl.with_(seed=wl.seed + 1000 * rank)
+    # inputs: this rank's own sequence
+    wl_r = rank_workload(wl, rank)
     qh, kh, vh = W.generate(wl_r)
     pin = [torch.from_numpy(x).view(torch.bfloat16).pin_memory() for x in (qh, kh, vh)]
     q, k, v = [x.to(dev, non_blocking=True) for x in pin]
@@ -247,7 +265,7 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
         b.record(stream)
         torch.cuda.synchronize()
         barrier()
-        return max_over_ranks(a.elapsed_time(b) / n)
+        return rank_max(a.elapsed_time(b) / n)
 
     for _ in range(args.warmup):
         forward()
@@ -269,7 +287,7 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
         if it >= args.warmup:
             for i, n in enumerate(stage_names):
                 per_stage[n].append(evs[i].elapsed_time(evs[i + 1]))
-    stage_ms = {n: max_over_ranks(statistics.mean(v)) for n, v in per_stage.items()}
+    stage_ms = {n: rank_max(statistics.mean(v)) for n, v in per_stage.items()}
 
     # ---- dense baselines on the same tensors
     od = torch.empty_like(q)
@@ -324,7 +342,7 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
     stage_roof = {n: {"GB/s": b / (stage_ms[n] * 1e-3) / 1e9, "frac_hbm": b / (stage_ms[n] * 1e-3) / 1e9 / hbm}
                   for n, b in stage_bytes.items()}
 
-    value = world * dense_flops(wl) / (ms * 1e-3) / 1e12
+    value = job_value(wl, world, ms)
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
         s = oracle_sample(wl, args.tau)
@@ -344,7 +362,7 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
         "stage_ms": stage_ms, "stage_hbm": stage_roof,
         "overhead_frac": (sum(stage_ms.values()) - attn_ms) / attn_ms,
         "roofline": roof, "cpu_baseline": cpu,
-        "e2e": {"value": world * dense_flops(wl) / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
+        "e2e": {"value": job_value(wl, world, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": KERNELS_PER_FORWARD * args.steps, "clocks": clocks,
     }
