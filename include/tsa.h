@@ -176,6 +176,27 @@ tsa_status tsa_forward(const tsa_params* p, const void* q, const void* k, const 
                        float* scores_out, int32_t* idx_out, int32_t* k_seq_out,
                        void* ws, size_t ws_bytes, void* stream);
 
+/* Proxy scores with no device allocation at all.  No counterpart on the
+ * pages: an addition for callers that cannot call cudaMalloc (a plug-in whose
+ * host framework owns every device allocation, code under a hard device
+ * memory budget, a C caller without an allocator for a workspace).
+ *
+ * Computes exactly what tsa_score computes, with the same kernels; the
+ * scratch that tsa_score takes from ws lives instead in a fixed array of
+ * TSA_NOALLOC_SCRATCH_BYTES inside the library, which every GPU that loads
+ * the library holds until the process exits.  The caller still passes q, k
+ * and scores.  Sizes whose scratch (tsa_stage_workspace_size) exceeds the
+ * array are rejected with TSA_ERR_WORKSPACE before any work is enqueued.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture.  All calls share the one array and it keeps the last call's
+ * contents: calls whose kernels overlap on the GPU (different streams, or
+ * different host threads on one device) race and must be serialised by the
+ * caller.  Calls no cudaMalloc, cudaFree or allocating library routine. */
+#define TSA_NOALLOC_SCRATCH_BYTES (16u << 20)
+tsa_status tsa_score_noalloc(const tsa_params* p, const void* q, const void* k, float* scores,
+                             void* stream);
+
 #ifdef __cplusplus
 }
 #endif

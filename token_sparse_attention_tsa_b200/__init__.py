@@ -28,7 +28,7 @@ DEVFLAG_NONFINITE, DEVFLAG_TIMEOUT, DEVFLAG_BAD_INDEX = 0x1, 0x2, 0x4
 EXPORTED = ("tsa_abi_version", "tsa_status_string", "tsa_check_params", "tsa_workspace_size",
             "tsa_stage_workspace_size", "tsa_reset_device_status", "tsa_get_device_status",
             "tsa_score", "tsa_budget", "tsa_select", "tsa_gather_qkv", "tsa_attend",
-            "tsa_attend_dense", "tsa_scatter", "tsa_forward")
+            "tsa_attend_dense", "tsa_scatter", "tsa_forward", "tsa_score_noalloc")
 
 
 class TSAError(RuntimeError):
@@ -82,6 +82,7 @@ def load(path: str | None = None):
             "tsa_attend_dense": ([_P, _v, _v, _v, _v, _v, _v, _sz, _v], ctypes.c_int),
             "tsa_scatter": ([_P, _v, _v, _v, _v, _v, _sz, _v], ctypes.c_int),
             "tsa_forward": ([_P, _v, _v, _v, _v, _v, _v, _v, _v, _sz, _v], ctypes.c_int),
+            "tsa_score_noalloc": ([_P, _v, _v, _v, _v], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             fn = getattr(lib, name)
@@ -174,6 +175,18 @@ def tsa_score(p, q, k, scores, ws, stream=None):
     _check(load().tsa_score(ctypes.byref(p), _ptr(q, "q", torch.bfloat16), _ptr(k, "k", torch.bfloat16),
                             _ptr(scores, "scores", torch.float32), _ptr(ws, "ws"), _nbytes(ws),
                             _stream(stream)), "tsa_score")
+
+
+NOALLOC_SCRATCH_BYTES = 16 << 20
+
+
+def tsa_score_noalloc(p, q, k, scores, stream=None):
+    """tsa_score for callers that cannot allocate device memory: no workspace;
+    the library's fixed 16 MiB device scratch is used instead (one call at a
+    time per device; the first call on a device must precede stream capture)."""
+    import torch
+    _check(load().tsa_score_noalloc(ctypes.byref(p), _ptr(q, "q", torch.bfloat16), _ptr(k, "k", torch.bfloat16),
+                                    _ptr(scores, "scores", torch.float32), _stream(stream)), "tsa_score_noalloc")
 
 
 def tsa_budget(p, scores, k_head, k_seq, ws, stream=None):

@@ -454,3 +454,51 @@ tsa_status tsa_forward(const tsa_params* p, const void* q, const void* k, const 
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Proxy scores without any device allocation.
+//
+// Some callers cannot call cudaMalloc: plug-ins whose host framework owns
+// every device allocation through its own pool, code with a hard device
+// memory budget, or plain C callers with no allocator for a workspace.  For
+// them tsa_score_noalloc runs the same score kernels as tsa_score with their
+// scratch (the per-chunk row statistics) in the fixed array below instead of
+// a caller workspace.  The array lives in the library's device image, so
+// every GPU that loads the library holds it until the process exits.
+namespace {
+
+static __device__ __align__(256) unsigned char g_score_scratch[TSA_NOALLOC_SCRATCH_BYTES];
+
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_score_scratch on the current device.  In host code the
+// array's name is only a host-side stand-in, so the address is looked up once
+// per device with that device current.
+tsa_status scratch_address(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TSA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_score_scratch) != cudaSuccess || !ptr) return TSA_ERR_CUDA;
+    g_scratch_ptr[dev] = ptr;
+  }
+  *out = g_scratch_ptr[dev];
+  return TSA_OK;
+}
+
+}  // namespace
+
+extern "C" tsa_status tsa_score_noalloc(const tsa_params* p, const void* q, const void* k, float* scores,
+                                        void* stream) {
+  tsa_status s = tsa_check_params(p);
+  if (s != TSA_OK) return s;
+  if (!tensors_ok({q, k, scores})) return TSA_ERR_INVALID_ARG;
+  if (layout_of(p).stage_end > static_cast<size_t>(TSA_NOALLOC_SCRATCH_BYTES)) return TSA_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  if ((s = scratch_address(&scratch)) != TSA_OK) return s;
+  // Every scratch entry the kernels read is written earlier in the same call,
+  // so nothing has to be cleared between calls.
+  return run_score(p, q, k, scores, scratch, static_cast<cudaStream_t>(stream));
+}
