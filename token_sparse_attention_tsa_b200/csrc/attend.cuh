@@ -9,16 +9,8 @@
 // applies).  With the identity selection the same kernel is the dense
 // baseline.
 //
-// One CTA computes one 128-row query tile of one head.  Warp roles:
-//   warp 0      TMA producer: Q tile once, then K/V tiles into a 2-stage ring
-//   warp 1      TMEM allocator and single-thread tcgen05.mma issuer
-//   warps 2..5  softmax: one thread per query row (TMEM lane), online softmax
-//               with lazy rescaling, P written to shared memory as bf16,
-//               epilogue normalises O and stores it.
-// TMEM columns: S double buffer [0,128) and [128,256), O [256, 256+D).
-// S = Q K^T and O += P V are kind::f16 MMAs (bf16 in, fp32 accumulate),
-// M = 128, operands in 128-byte-swizzled shared memory.
-//
+// Two 128-row query tiles of one head per CTA, warp-specialised (see the
+// comment above attend2_kernel for the roles, TMEM plan and MMA order).
 // Every wait is bounded (WaitCtl); a timeout sets the device status word,
 // the CTA drains its in-flight copies/MMAs, frees TMEM and returns.
 #pragma once
@@ -28,29 +20,6 @@
 #include "sm100.cuh"
 
 namespace tsa {
-
-template <int D>
-struct AttnLayout {
-  static constexpr int BM = 128;                 // query rows per CTA
-  static constexpr int BN = 128;                 // keys per KV tile
-  static constexpr int NS = 2;                   // K/V pipeline stages
-  static constexpr int CHUNK = 128 * 128;        // one 128-row x 64-col bf16 SW128 block
-  static constexpr int NCH = D / 64;             // 64-column chunks of a row
-  static constexpr int Q_BYTES = BM * D * 2;
-  static constexpr int KV_BYTES = BN * D * 2;
-  static constexpr int P_BYTES = BM * BN * 2;
-  static constexpr int OFF_Q = 0;
-  static constexpr int OFF_K = OFF_Q + Q_BYTES;
-  static constexpr int OFF_V = OFF_K + NS * KV_BYTES;
-  static constexpr int OFF_P = OFF_V + NS * KV_BYTES;
-  static constexpr int OFF_BAR = OFF_P + P_BYTES;
-  static constexpr int TOTAL = OFF_BAR + 256;
-  // +1 KiB for aligning the base to 1024 B; padded so only one CTA fits per
-  // SM (each CTA allocates all 512 TMEM columns).
-  static constexpr int ALLOC = (TOTAL + 1024) > 120 * 1024 ? (TOTAL + 1024) : 120 * 1024;
-  static constexpr int TMEM_COLS = 512;
-  static constexpr int TMEM_O = 256;
-};
 
 struct AttnArgs {
   const int32_t* k_seq;   // valid rows per sequence (null: L)
@@ -67,24 +36,70 @@ struct AttnArgs {
   uint64_t limit_ns;      // per-wait time limit
 };
 
-enum : int {
-  BAR_Q = 0,
-  BAR_KFULL = 1,   // +stage
-  BAR_VFULL = 3,   // +stage
-  BAR_KVEMPTY = 5, // +stage
-  BAR_SFULL = 7,   // +buffer
-  BAR_SFREE = 9,   // +buffer
-  BAR_PFULL = 11,
-  BAR_PVDONE = 12,
-  BAR_DRAIN = 13,
-  BAR_COUNT = 14
+// ---------------------------------------------------------------------------
+// Two query tiles per CTA (rows [256c, 256c+256) of one head), ping-ponged,
+// with two softmax warpgroups per tile:
+//   warps 0..7   softmax of query tile 0 (warps 0..3 columns 0..63 of every
+//                row, warps 4..7 columns 64..127)
+//   warps 8..15  softmax of query tile 1 (same split)
+//   warp 16      TMEM allocator + MMA issuer
+//   warp 17      TMA producer
+// Each row's max and sum are combined across its two halves through shared
+// memory behind a named barrier of the tile's 256 threads; the barrier also
+// ANDs the threads' progress flags, so both halves always take the same
+// branch (a timed-out wait can never leave one half at a barrier alone).
+// TMEM: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D, 256+2D).  Each
+// half writes its 64 P values (bf16, two per 32-bit column) over the first 32
+// of its own 64 S columns, and the P.V MMA reads P from TMEM (k-steps 0..3
+// from the first half's columns, 4..7 from the second's), so P never touches
+// shared memory.  The softmax reads S twice (row max first, then the
+// exponentials), keeping only 32 values in registers at a time.  K and V
+// tiles stream through one TMA ring of NSLOT slots in the order K0 V0 K1 V1 ...
+// Per KV tile j the MMA warp issues S0_j, PV1_{j-1}, S1_j, PV0_j: while one
+// tile's softmax runs the tensor core works on the other tile.  S0_{j+1}
+// overwrites the columns P0_j is read from by PV0_j, issued just before it by
+// the same thread; tcgen05.mma ops of one thread execute in issue order, so
+// the read precedes the overwrite (the same reliance as the open CUTLASS
+// sm100 attention mainloop).
+template <int D, int PARTS>
+struct Attn2Layout {
+  static constexpr int BM = 128;
+  static constexpr int BN = 128;
+  static constexpr int SOFT_WARPS = 8 * PARTS;        // 4 warps per part per tile
+  static constexpr int COLS = BN / PARTS;              // S columns per softmax thread
+  static constexpr int THREADS = (SOFT_WARPS + 2) * 32;
+  static constexpr int MMA_WARP = SOFT_WARPS;
+  static constexpr int LOAD_WARP = SOFT_WARPS + 1;
+  static constexpr int CHUNK = 128 * 128;            // 128 rows x 64 bf16 columns, SW128
+  static constexpr int NCH = D / 64;
+  static constexpr int TILE = 128 * D * 2;            // bytes of one Q, K or V tile
+  static constexpr int NSLOT = D == 128 ? 4 : 9;      // K/V ring slots
+  static constexpr int OFF_Q0 = 0;
+  static constexpr int OFF_Q1 = TILE;
+  static constexpr int OFF_RING = 2 * TILE;
+  static constexpr int OFF_X = OFF_RING + NSLOT * TILE;        // row max / sum exchange
+  static constexpr int X_BYTES = 2 * 2 * 2 * 128 * 4;          // [parity][tile][half][row]
+  static constexpr int OFF_BAR = OFF_X + X_BYTES;
+  static constexpr int TOTAL = OFF_BAR + 512;
+  static constexpr int ALLOC = (TOTAL + 1024) > 120 * 1024 ? (TOTAL + 1024) : 120 * 1024;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int TMEM_O = 256;
+  // barrier indices
+  static constexpr int B_Q = 0;
+  static constexpr int B_FULL = 1;                    // + slot
+  static constexpr int B_EMPTY = 1 + NSLOT;           // + slot
+  static constexpr int B_S = 1 + 2 * NSLOT;           // + tile (S ready)
+  static constexpr int B_P = B_S + 2;                 // + tile (P written)
+  static constexpr int B_PV = B_P + 2;                // + tile (P.V complete)
+  static constexpr int B_DRAIN = B_PV + 2;
+  static constexpr int B_COUNT = B_DRAIN + 1;
 };
 
-template <int D>
-__global__ void __launch_bounds__(192, 1)
-    attend_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                  const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
-  using C = AttnLayout<D>;
+template <int D, int PARTS>
+__global__ void __launch_bounds__(Attn2Layout<D, PARTS>::THREADS, 1)
+    attend2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                   const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
+  using C = Attn2Layout<D, PARTS>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -94,37 +109,39 @@ __global__ void __launch_bounds__(192, 1)
   const int bh = blockIdx.y;
   const int b = bh / a.Hq;
   const int h = bh - b * a.Hq;
-  const int t = a.n_tiles - 1 - static_cast<int>(blockIdx.x);  // longest tiles first
+  const int n_pairs = (a.n_tiles + 1) >> 1;
+  const int t0 = 2 * (n_pairs - 1 - static_cast<int>(blockIdx.x));  // longest pairs first
 
   int valid = a.k_seq ? a.k_seq[b] : a.L;
   valid = valid < 0 ? 0 : (valid > a.L ? a.L : valid);
-  if (t * C::BM >= valid) return;  // uniform over the CTA, before any barrier
-  const int n_kv = t + 1;           // causal: KV tiles 0..t
+  if (t0 * C::BM >= valid) return;                 // uniform, before any barrier
+  const bool two = (t0 + 1) * C::BM < valid;       // second query tile has rows
+  const int last0 = t0;                            // tile 0 attends KV tiles 0..t0
+  const int n_kv = two ? t0 + 2 : t0 + 1;          // tile 1 attends 0..t0+1
 
   auto bar = [&](int i) -> uint32_t { return base + C::OFF_BAR + 8u * static_cast<uint32_t>(i); };
-  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + C::OFF_BAR + 8 * BAR_COUNT);
-  volatile int* cta_abort = reinterpret_cast<volatile int*>(gbase + C::OFF_BAR + 8 * BAR_COUNT + 4);
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + C::OFF_BAR + 8 * C::B_COUNT);
+  volatile int* cta_abort = reinterpret_cast<volatile int*>(gbase + C::OFF_BAR + 8 * C::B_COUNT + 4);
+  auto slot_of = [](int n) { return n % C::NSLOT; };
+  auto use_of = [](int n) { return n / C::NSLOT; };
+  auto ring = [&](int n) -> uint32_t { return base + C::OFF_RING + slot_of(n) * C::TILE; };
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(BAR_Q), 1);
-    for (int s = 0; s < C::NS; ++s) {
-      mbar_init(bar(BAR_KFULL + s), 1);
-      mbar_init(bar(BAR_VFULL + s), 1);
-      mbar_init(bar(BAR_KVEMPTY + s), 1);
+    mbar_init(bar(C::B_Q), 1);
+    for (int s = 0; s < C::NSLOT; ++s) {
+      mbar_init(bar(C::B_FULL + s), 1);
+      mbar_init(bar(C::B_EMPTY + s), 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(bar(BAR_SFULL + s), 1);
-      mbar_init(bar(BAR_SFREE + s), 128);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(C::B_S + t), 1);
+      mbar_init(bar(C::B_P + t), 128 * PARTS);
+      mbar_init(bar(C::B_PV + t), 1);
     }
-    mbar_init(bar(BAR_PFULL), 128);
-    mbar_init(bar(BAR_PVDONE), 1);
-    mbar_init(bar(BAR_DRAIN), 1);
-    // another CTA of this launch already timed out: skip the work (still
-    // tear down cleanly)
+    mbar_init(bar(C::B_DRAIN), 1);
     *cta_abort = (a.abort_word && *reinterpret_cast<volatile uint32_t*>(a.abort_word)) ? 1 : 0;
     fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == C::MMA_WARP) {
     tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -135,199 +152,274 @@ __global__ void __launch_bounds__(192, 1)
   const WaitCtl wc{cta_abort, a.status, a.abort_word, a.limit_ns};
   const bool run = (*cta_abort == 0);
 
-  if (warp == 0) {
+  if (warp == C::LOAD_WARP) {
     // ------------------------------------------------------------ producer
-    if (lane == 0 && run) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
-      const int zq = bh;
-      const int zkv = b * a.Hkv_map + h / a.G_map;
-      mbar_arrive_expect_tx(bar(BAR_Q), C::Q_BYTES);
-#pragma unroll
-      for (int c = 0; c < C::NCH; ++c)
-        tma_load_3d(base + C::OFF_Q + c * C::CHUNK, &tmQ, bar(BAR_Q), c * 64, t * C::BM, zq);
-      int issued = 0;
-      for (int j = 0; j < n_kv; ++j) {
-        const int s = j % C::NS;
-        const int n = j / C::NS;
-        if (j >= C::NS && !mbar_wait(bar(BAR_KVEMPTY + s), (n - 1) & 1, wc)) break;
-        mbar_arrive_expect_tx(bar(BAR_KFULL + s), C::KV_BYTES);
-#pragma unroll
-        for (int c = 0; c < C::NCH; ++c)
-          tma_load_3d(base + C::OFF_K + s * C::KV_BYTES + c * C::CHUNK, &tmK, bar(BAR_KFULL + s),
-                      c * 64, j * C::BN, zkv);
-        mbar_arrive_expect_tx(bar(BAR_VFULL + s), C::KV_BYTES);
-#pragma unroll
-        for (int c = 0; c < C::NCH; ++c)
-          tma_load_3d(base + C::OFF_V + s * C::KV_BYTES + c * C::CHUNK, &tmV, bar(BAR_VFULL + s),
-                      c * 64, j * C::BN, zkv);
-        issued = j + 1;
+    // The whole warp runs the loop (uniform values); one elected lane issues.
+    if (run) {
+      const bool leader = elect_one();
+      if (leader) {
+        tma_prefetch_desc(&tmQ);
+        tma_prefetch_desc(&tmK);
+        tma_prefetch_desc(&tmV);
       }
-      if (*cta_abort) {  // let every copy still in flight land before exit
-        mbar_wait_drain(bar(BAR_Q), 0, 1000000000ull);
-        for (int j = issued - C::NS < 0 ? 0 : issued - C::NS; j < issued; ++j) {
-          mbar_wait_drain(bar(BAR_KFULL + j % C::NS), (j / C::NS) & 1, 1000000000ull);
-          mbar_wait_drain(bar(BAR_VFULL + j % C::NS), (j / C::NS) & 1, 1000000000ull);
+      const int zkv = b * a.Hkv_map + h / a.G_map;
+      if (leader) {
+        mbar_arrive_expect_tx(bar(C::B_Q), (two ? 2 : 1) * C::TILE);
+#pragma unroll
+        for (int c = 0; c < C::NCH; ++c) {
+          tma_load_3d(base + C::OFF_Q0 + c * C::CHUNK, &tmQ, bar(C::B_Q), c * 64, t0 * C::BM, bh);
+          if (two) tma_load_3d(base + C::OFF_Q1 + c * C::CHUNK, &tmQ, bar(C::B_Q), c * 64, (t0 + 1) * C::BM, bh);
         }
       }
+      int issued = 0;
+      for (int n = 0; n < 2 * n_kv; ++n) {
+        const int s = slot_of(n), u = use_of(n);
+        if (u >= 1 && !__all_sync(0xffffffffu, mbar_wait(bar(C::B_EMPTY + s), (u - 1) & 1, wc))) break;
+        if (leader) {
+          mbar_arrive_expect_tx(bar(C::B_FULL + s), C::TILE);
+          const CUtensorMap* m = (n & 1) ? &tmV : &tmK;
+#pragma unroll
+          for (int c = 0; c < C::NCH; ++c)
+            tma_load_3d(ring(n) + c * C::CHUNK, m, bar(C::B_FULL + s), c * 64, (n >> 1) * C::BN, zkv);
+        }
+        issued = n + 1;
+      }
+      if (leader && *cta_abort) {  // let every copy still in flight land before exit
+        mbar_wait_drain(bar(C::B_Q), 0, 1000000000ull);
+        for (int n = issued - C::NSLOT < 0 ? 0 : issued - C::NSLOT; n < issued; ++n)
+          mbar_wait_drain(bar(C::B_FULL + slot_of(n)), use_of(n) & 1, 1000000000ull);
+      }
     }
-  } else if (warp == 1) {
+  } else if (warp == C::MMA_WARP) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && run) {
+    // The whole warp runs the loop so loop state and descriptors are uniform;
+    // one elected lane issues every MMA and commit.  Descriptors are built
+    // once; a k-step only adds its byte offset >> 4 to the start-address
+    // field (shared-memory addresses stay below 2^18, so the field never
+    // carries over).
+    if (run) {
+      const bool leader = elect_one();
       constexpr uint32_t idS = idesc_bf16_f32(128, C::BN, 0, 0);
       constexpr uint32_t idO = idesc_bf16_f32(128, D, 0, 1);
-      bool ok = mbar_wait(bar(BAR_Q), 0, wc);
-      for (int j = 0; ok && j <= n_kv; ++j) {
-        if (j < n_kv) {
-          const int sb = j & 1;
-          const int s = j % C::NS;
-          if (j >= 2 && !(ok = mbar_wait(bar(BAR_SFREE + sb), ((j >> 1) - 1) & 1, wc))) break;
-          if (!(ok = mbar_wait(bar(BAR_KFULL + s), (j / C::NS) & 1, wc))) break;
-          tc_fence_after();
+      const uint64_t dq0 = smem_desc(base + C::OFF_Q0, 16, 1024, kSwizzle128B);
+      const uint64_t dq1 = smem_desc(base + C::OFF_Q1, 16, 1024, kSwizzle128B);
+      const uint64_t dk0 = smem_desc(base + C::OFF_RING, 16, 1024, kSwizzle128B);
+      const uint64_t dv0 = smem_desc(base + C::OFF_RING, C::CHUNK, 1024, kSwizzle128B);
+      auto issue_s = [&](int t, int j) {
+        const uint64_t dq = t ? dq1 : dq0;
+        const uint64_t dk = dk0 + static_cast<uint64_t>((slot_of(2 * j) * C::TILE) >> 4);
+        if (leader) {
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-            mma_bf16_ss(tmem + sb * 128, smem_desc(base + C::OFF_Q + off, 16, 1024, kSwizzle128B),
-                        smem_desc(base + C::OFF_K + s * C::KV_BYTES + off, 16, 1024, kSwizzle128B),
-                        idS, kk > 0 ? 1u : 0u);
+            const uint64_t off = static_cast<uint64_t>(((kk >> 2) * C::CHUNK + (kk & 3) * 32) >> 4);
+            mma_bf16_ss(tmem + t * 128, dq + off, dk + off, idS, kk > 0 ? 1u : 0u);
           }
-          mma_commit(bar(BAR_SFULL + sb));
+          mma_commit(bar(C::B_S + t));
         }
-        if (j >= 1) {
-          const int jj = j - 1;
-          const int s = jj % C::NS;
-          if (!(ok = mbar_wait(bar(BAR_PFULL), jj & 1, wc))) break;
-          if (!(ok = mbar_wait(bar(BAR_VFULL + s), (jj / C::NS) & 1, wc))) break;
-          tc_fence_after();
+      };
+      auto issue_pv = [&](int t, int j) {
+        const uint64_t dv = dv0 + static_cast<uint64_t>((slot_of(2 * j + 1) * C::TILE) >> 4);
+        if (leader) {
 #pragma unroll
           for (int kk = 0; kk < C::BN / 16; ++kk) {
-            const uint32_t pa = (kk >> 2) * C::CHUNK + (kk & 3) * 32;
-            mma_bf16_ss(tmem + C::TMEM_O, smem_desc(base + C::OFF_P + pa, 16, 1024, kSwizzle128B),
-                        smem_desc(base + C::OFF_V + s * C::KV_BYTES + kk * 2048, C::CHUNK, 1024,
-                                  kSwizzle128B),
-                        idO, (jj > 0 || kk > 0) ? 1u : 0u);
+            // P of keys [16kk, 16kk+16): part p = 16kk / COLS holds them from
+            // column p*COLS, two keys per column.
+            const uint32_t pcol = (16 * kk / C::COLS) * C::COLS + (16 * kk % C::COLS) / 2;
+            mma_bf16_ts(tmem + C::TMEM_O + t * D, tmem + t * 128 + pcol,
+                        dv + static_cast<uint64_t>((kk * 2048) >> 4), idO, (j > 0 || kk > 0) ? 1u : 0u);
           }
-          mma_commit(bar(BAR_PVDONE));
-          mma_commit(bar(BAR_KVEMPTY + s));
+          mma_commit(bar(C::B_PV + t));
         }
-      }
-      // all issued MMAs complete before TMEM is released
-      mma_commit(bar(BAR_DRAIN));
-      mbar_wait_drain(bar(BAR_DRAIN), 0, 1000000000ull);
-    }
-  } else if (run) {
-    // ------------------------------------------------------------ softmax
-    const int q4 = warp & 3;
-    const int r = q4 * 32 + lane;                       // row within the tile
-    const int row = t * C::BM + r;                      // compressed row index
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(q4 * 32) << 16);
-    const float sl2 = a.scale_log2;
-    float m_used = -INFINITY;                           // running max (log2 units)
-    float l = 0.f;
-    bool ok = true;
-    for (int j = 0; j < n_kv; ++j) {
-      const int sb = j & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(BAR_SFULL + sb), (j >> 1) & 1, wc));
-      if (!ok) break;
-      tc_fence_after();
-      float sv[4][32];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(lane_base + sb * 128 + c * 32, sv[c]);
-      tmem_ld_wait();
-      tc_fence_before();
-      mbar_arrive(bar(BAR_SFREE + sb));
-
-      const bool diag = (j == n_kv - 1);
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          if (diag && (c * 32 + e) > r) sv[c][e] = -INFINITY;
-          mx = fmaxf(mx, sv[c][e]);
-        }
-      const float m_new = fmaxf(m_used, mx * sl2);
-      const bool resc = m_new > m_used + 8.0f;         // lazy rescale (factor <= 2^8 tolerated)
-
-      if (j > 0) {
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(BAR_PVDONE), (j - 1) & 1, wc));
-        if (!ok) break;
+      };
+      auto commit_to = [&](uint32_t br) {
+        if (leader) mma_commit(br);
+      };
+      auto wait_all = [&](uint32_t br, uint32_t par) {
+        return __all_sync(0xffffffffu, mbar_wait(br, par, wc));
+      };
+      auto full = [&](int n) { return wait_all(bar(C::B_FULL + slot_of(n)), use_of(n) & 1); };
+      bool ok = wait_all(bar(C::B_Q), 0);
+      for (int j = 0; ok && j < n_kv; ++j) {
+        if (!(ok = full(2 * j))) break;                                  // K_j
         tc_fence_after();
-        if (__any_sync(0xffffffffu, resc)) {
-          const float alpha = resc ? ex2_approx(m_used - m_new) : 1.f;
-          l *= alpha;
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            float ov[32];
-            tmem_ld32(lane_base + C::TMEM_O + c * 32, ov);
-            tmem_ld_wait();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) ov[e] *= alpha;
-            tmem_st32(lane_base + C::TMEM_O + c * 32, ov);
-          }
-          tmem_st_wait();
+        if (j <= last0) issue_s(0, j);
+        if (two && j >= 1) {
+          if (!(ok = wait_all(bar(C::B_P + 1), (j - 1) & 1))) break;
+          tc_fence_after();
+          issue_pv(1, j - 1);
+          commit_to(bar(C::B_EMPTY + slot_of(2 * j - 1)));               // V_{j-1} done
+        }
+        if (two) issue_s(1, j);
+        commit_to(bar(C::B_EMPTY + slot_of(2 * j)));                     // K_j done
+        if (j <= last0) {
+          if (!(ok = wait_all(bar(C::B_P + 0), j & 1))) break;
+          if (!(ok = full(2 * j + 1))) break;                            // V_j
+          tc_fence_after();
+          issue_pv(0, j);
+          if (!two) commit_to(bar(C::B_EMPTY + slot_of(2 * j + 1)));
         }
       }
+      if (ok && two) {
+        const int j = n_kv - 1;
+        if (wait_all(bar(C::B_P + 1), j & 1) && full(2 * j + 1)) {
+          tc_fence_after();
+          issue_pv(1, j);
+          commit_to(bar(C::B_EMPTY + slot_of(2 * j + 1)));
+        }
+      }
+      commit_to(bar(C::B_DRAIN));
+      if (leader) mbar_wait_drain(bar(C::B_DRAIN), 0, 1000000000ull);
+    }
+  } else if (run && (warp < C::SOFT_WARPS / 2 || two)) {
+    // ------------------------------------------------------------ softmax
+    const int tt = warp / (4 * PARTS);           // query tile of this warp
+    const int half = (warp >> 2) % PARTS;        // columns [COLS*half, COLS*half+COLS)
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;                // row within the tile
+    const int tile = t0 + tt;
+    const int row = tile * C::BM + r;
+    const int last = tile;                       // its diagonal KV tile
+    const bool last_active = tt == (two ? 1 : 0);
+    const uint32_t named = 1 + tt;               // named barrier of the tile's 256 threads
+    const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
+    const uint32_t s_col = tmem + lane_off + tt * 128 + half * C::COLS;
+    const uint32_t p_col = s_col;                // P over the first COLS/2 of the part's columns
+    const uint32_t o_col = tmem + lane_off + C::TMEM_O + tt * D + half * (D / PARTS);
+    float* xch = reinterpret_cast<float*>(gbase + C::OFF_X);   // [parity][tile][half][row]
+    auto xidx = [&](int par, int hf) { return ((par * 2 + tt) * 2 + hf) * 128 + r; };
+    const float sl2 = a.scale_log2;
+    float m_used = -INFINITY;
+    float l = 0.f;                               // this half's share of the row sum
+    bool live = true;
+    for (int j = 0; j <= last; ++j) {
+      live = live && __all_sync(0xffffffffu, mbar_wait(bar(C::B_S + tt), j & 1, wc));
+      float mh = -INFINITY;
+      const bool diag = (j == last);
+      if (live) {  // pass 1: this part's row max
+        tc_fence_after();
+        constexpr int NC = C::COLS / 32;
+        float sv[NC][32];
+#pragma unroll
+        for (int c = 0; c < NC; ++c) tmem_ld32(s_col + c * 32, sv[c]);
+        tmem_ld_wait();
+        if (diag) {  // causal mask, only on the diagonal tile
+#pragma unroll
+          for (int c = 0; c < NC; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if ((half * C::COLS + c * 32 + e) > r) sv[c][e] = -INFINITY;
+        }
+        float m8[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) m8[u] = sv[0][u];
+#pragma unroll
+        for (int c = 0; c < NC; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (c > 0 || e >= 8) m8[e & 7] = fmaxf(m8[e & 7], sv[c][e]);
+        mh = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+      }
+      float mx = mh;
+      if constexpr (PARTS == 2) {
+        xch[xidx(j & 1, half)] = mh;
+        live = bar_and(named, 256, live);        // both halves agree to go on
+        if (!live) continue;                     // keep the barrier count uniform
+        mx = fmaxf(mh, xch[xidx(j & 1, half ^ 1)]);
+      } else {
+        if (!live) continue;
+      }
+      const float m_new = fmaxf(m_used, mx * sl2);
+      const bool resc = m_new > m_used + 8.0f;   // lazy rescale (factor <= 2^8 tolerated)
+      const float alpha = resc ? ex2_approx(m_used - m_new) : 1.f;
       if (resc) m_used = m_new;
-
-      // P = exp2(s * scale_log2 - m_used) in bf16, row r of a K-major SW128 tile
       const float nm = -m_used;
-      float rs = 0.f;
-      uint8_t* prow = gbase + C::OFF_P + (r >> 3) * 1024 + (r & 7) * 128;
+      float r8[8];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int u = 0; u < 8; ++u) r8[u] = 0.f;
+      // pass 2: S columns [32c, 32c+32) of the part give P columns
+      // [16c, 16c+16), which lie in columns already read.
 #pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          float pv[8];
+      for (int c = 0; c < C::COLS / 32; ++c) {
+        float sv[32];
+        tmem_ld32(s_col + c * 32, sv);
+        tmem_ld_wait();
+        if (diag) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            pv[e] = ex2_approx(fmaf(sv[c][g * 8 + e], sl2, nm));
-            rs += pv[e];
+          for (int e = 0; e < 32; ++e)
+            if ((half * C::COLS + c * 32 + e) > r) sv[e] = -INFINITY;
+        }
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float p0 = ex2_approx(fmaf(sv[2 * e], sl2, nm));
+          const float p1 = ex2_approx(fmaf(sv[2 * e + 1], sl2, nm));
+          r8[e & 7] += p0 + p1;
+          pk[e] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16u(p_col + c * 16, pk);
+      }
+      l = l * alpha + (((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7])));
+      // O is rescaled only when a row's max grew past the lazy threshold, and
+      // then only once the previous P.V into O has completed (and before this
+      // tile's P.V, which waits for P_FULL).  Otherwise the wait is skipped:
+      // P.V MMAs into one accumulator run in issue order.  The PV barrier can
+      // never be two phases ahead here (P.V j needs this tile's P first), so a
+      // parity wait after skipped ones still names the right phase.
+      if (j > 0 && __any_sync(0xffffffffu, resc)) {
+        live = __all_sync(0xffffffffu, mbar_wait(bar(C::B_PV + tt), (j - 1) & 1, wc));
+        if (live) {
+          tc_fence_after();
+          {
+#pragma unroll
+            for (int c = 0; c < D / PARTS / 32; ++c) {
+              float ov[32];
+              tmem_ld32(o_col + c * 32, ov);
+              tmem_ld_wait();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) ov[e] *= alpha;
+              tmem_st32(o_col + c * 32, ov);
+            }
           }
-          const int ch = c * 4 + g;                     // 16-byte chunk 0..15 of the row
-          const int blk = ch >> 3;                      // 64-column block
-          const int cc = (ch & 7) ^ (r & 7);            // 128B swizzle
-          uint4 pk;
-          pk.x = pack_bf16x2(pv[0], pv[1]);
-          pk.y = pack_bf16x2(pv[2], pv[3]);
-          pk.z = pack_bf16x2(pv[4], pv[5]);
-          pk.w = pack_bf16x2(pv[6], pv[7]);
-          *reinterpret_cast<uint4*>(prow + blk * C::CHUNK + cc * 16) = pk;
         }
       }
-      l += rs;
-
-      // Rows of the last KV tile at or beyond `valid` may hold any bits; their
-      // P weights are 0 but 0 * NaN would poison O, so zero them in smem.
-      if (diag && (j * C::BN + C::BN > valid)) {
-        const int s = j % C::NS;
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(BAR_VFULL + s), (j / C::NS) & 1, wc));
-        if (!ok) break;
-        if (j * C::BN + r >= valid) {
+      // Rows of the KV tile that holds `valid` may carry any bits beyond it;
+      // their P weights are 0 but 0 * NaN would poison O, so zero them.
+      if (live && half == 0 && diag && last_active && (j * C::BN + C::BN > valid)) {
+        const int n = 2 * j + 1;
+        live = __all_sync(0xffffffffu, mbar_wait(bar(C::B_FULL + slot_of(n)), use_of(n) & 1, wc));
+        if (live && j * C::BN + r >= valid) {
 #pragma unroll
           for (int c = 0; c < C::NCH; ++c) {
-            uint4* vrow = reinterpret_cast<uint4*>(gbase + C::OFF_V + s * C::KV_BYTES + c * C::CHUNK + r * 128);
+            uint4* vrow = reinterpret_cast<uint4*>(gbase + C::OFF_RING + slot_of(n) * C::TILE + c * C::CHUNK + r * 128);
 #pragma unroll
             for (int e = 0; e < 8; ++e) vrow[e] = make_uint4(0, 0, 0, 0);
           }
         }
+        fence_proxy_async_smem();
       }
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(bar(BAR_PFULL));
+      if (live) {
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(bar(C::B_P + tt));
+      }
     }
-
     // ------------------------------------------------------------ epilogue
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(BAR_PVDONE), (n_kv - 1) & 1, wc));
-    if (ok) {
+    live = live && __all_sync(0xffffffffu, mbar_wait(bar(C::B_PV + tt), last & 1, wc));
+    float lt = l;
+    if constexpr (PARTS == 2) {
+      xch[xidx(0, half)] = l;  // parity-0 slots are free: every read of them is behind us
+      live = bar_and(named, 256, live);
+      if (live) lt = l + xch[xidx(0, half ^ 1)];
+    }
+    if (live) {
       tc_fence_after();
-      const float inv_l = 1.f / l;
-      __nv_bfloat16* orow = a.o + (static_cast<size_t>(bh) * a.L + row) * D;
+      const float inv_l = 1.f / lt;
+      __nv_bfloat16* orow = a.o + (static_cast<size_t>(bh) * a.L + row) * D + half * (D / PARTS);
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < D / PARTS / 32; ++c) {
         float ov[32];
-        tmem_ld32(lane_base + C::TMEM_O + c * 32, ov);
+        tmem_ld32(o_col + c * 32, ov);
         tmem_ld_wait();
         if (row < valid) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
@@ -342,14 +434,14 @@ __global__ void __launch_bounds__(192, 1)
           }
         }
       }
-      if (a.lse && row < valid)
-        a.lse[static_cast<size_t>(bh) * a.L + row] = (m_used + __log2f(l)) * 0.69314718055994531f;
+      if (a.lse && half == 0 && row < valid)
+        a.lse[static_cast<size_t>(bh) * a.L + row] = (m_used + __log2f(lt)) * 0.69314718055994531f;
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == C::MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }

@@ -24,8 +24,6 @@
 
 namespace {
 
-using tsa::AttnLayout;
-
 constexpr size_t kAlign = 256;
 constexpr int kMaxDevices = 64;
 
@@ -131,6 +129,9 @@ bool ensure_smem(std::atomic<int> (&done)[kMaxDevices], K kernel, int bytes) {
 std::atomic<int> g_attn64[kMaxDevices], g_attn128[kMaxDevices], g_st64[kMaxDevices],
     g_st128[kMaxDevices], g_sum64[kMaxDevices], g_sum128[kMaxDevices], g_budget[kMaxDevices],
     g_select[kMaxDevices];
+
+// Softmax warpgroups per 128-row query tile in the attention kernel.
+constexpr int kSoftmaxParts = 2;
 
 constexpr int kBudgetSmem = tsa::BS_WARPS * 256 * (8 + 4);
 constexpr int kSelectSmem = tsa::BS_WARPS * 256 * 4;
@@ -261,15 +262,15 @@ tsa_status run_attend(const tsa_params* p, const void* q, const void* k, const v
   a.n_tiles = (p->L + 127) / 128;
   a.scale_log2 = scale_of(p) * 1.4426950408889634f;
   a.limit_ns = limit_ns_of(p);
-  const dim3 grid(a.n_tiles, bhq);
+  const dim3 grid((a.n_tiles + 1) / 2, bhq);  // two query tiles per CTA
   if (p->d == 128) {
-    constexpr int sm = AttnLayout<128>::ALLOC;
-    if (!ensure_smem(g_attn128, tsa::attend_kernel<128>, sm)) return TSA_ERR_CUDA;
-    tsa::attend_kernel<128><<<grid, 192, sm, st>>>(mq, mk, mv, a);
+    using L = tsa::Attn2Layout<128, kSoftmaxParts>;
+    if (!ensure_smem(g_attn128, tsa::attend2_kernel<128, kSoftmaxParts>, L::ALLOC)) return TSA_ERR_CUDA;
+    tsa::attend2_kernel<128, kSoftmaxParts><<<grid, L::THREADS, L::ALLOC, st>>>(mq, mk, mv, a);
   } else {
-    constexpr int sm = AttnLayout<64>::ALLOC;
-    if (!ensure_smem(g_attn64, tsa::attend_kernel<64>, sm)) return TSA_ERR_CUDA;
-    tsa::attend_kernel<64><<<grid, 192, sm, st>>>(mq, mk, mv, a);
+    using L = tsa::Attn2Layout<64, kSoftmaxParts>;
+    if (!ensure_smem(g_attn64, tsa::attend2_kernel<64, kSoftmaxParts>, L::ALLOC)) return TSA_ERR_CUDA;
+    tsa::attend2_kernel<64, kSoftmaxParts><<<grid, L::THREADS, L::ALLOC, st>>>(mq, mk, mv, a);
   }
   return launch_ok();
 }
