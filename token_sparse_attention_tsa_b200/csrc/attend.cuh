@@ -134,7 +134,7 @@ __global__ void __launch_bounds__(Attn2Layout<D, PARTS>::THREADS, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar(C::B_S + t), 1);
-      mbar_init(bar(C::B_P + t), 128 * PARTS);
+      mbar_init(bar(C::B_P + t), 4 * PARTS);      // one arrival per softmax warp
       mbar_init(bar(C::B_PV + t), 1);
     }
     mbar_init(bar(C::B_DRAIN), 1);
@@ -399,9 +399,12 @@ __global__ void __launch_bounds__(Attn2Layout<D, PARTS>::THREADS, 1)
         fence_proxy_async_smem();
       }
       if (live) {
+        // the warp's TMEM stores (and V zeroing) are complete; one lane
+        // arrives for the warp
         tmem_st_wait();
         tc_fence_before();
-        mbar_arrive(bar(C::B_P + tt));
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(C::B_P + tt));
       }
     }
     // ------------------------------------------------------------ epilogue

@@ -101,13 +101,13 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [heads, L, d] bf16 rows; box = 128 rows x 64 columns, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, int d, int L, int heads) {
+// [heads, L, d] bf16 rows; box = box_rows rows x 64 columns, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, int d, int L, int heads, int box_rows = 128) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(heads)};
   cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(L) * d * 2};
-  cuuint32_t box[3] = {64, 128, 1};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -140,39 +140,46 @@ constexpr int kSelectSmem = tsa::BS_WARPS * 256 * 4;
 tsa_status run_score(const tsa_params* p, const void* q, const void* k, float* scores, void* ws,
                      cudaStream_t st) {
   const WsLayout w = layout_of(p);
+  const int bhq = p->B * p->Hq;
+  CUtensorMap mq, mk;
+  if (!make_map(&mq, q, p->d, p->L, bhq, tsa::SC_ROWS) ||
+      !make_map(&mk, k, p->d, p->L, p->B * p->Hkv, tsa::SC_KEYS))
+    return TSA_ERR_CUDA;
   tsa::ScoreArgs a;
-  a.q = static_cast<const __nv_bfloat16*>(q);
-  a.k = static_cast<const __nv_bfloat16*>(k);
   a.scores = scores;
   a.part_m = at<float>(ws, w.part_m);
   a.part_z = at<double>(ws, w.part_z);
   a.stats = at<float2>(ws, w.stats);
+  a.status = at<uint32_t>(ws, 0);
+  a.abort_word = at<uint32_t>(ws, 8);
   a.L = p->L;
   a.w = p->w;
   a.Hq = p->Hq;
   a.Hkv = p->Hkv;
   a.G = p->Hq / p->Hkv;
   a.n_chunks = score_chunks(p);
-  a.scale = scale_of(p);
-  const int bhq = p->B * p->Hq;
-  const dim3 g1(a.n_chunks, bhq), g2((p->L + tsa::SC_KEYS - 1) / tsa::SC_KEYS, bhq);
-  const int sm1 = 2 * p->d * 128 * 4;
-  const int sm2 = sm1 + 16 * 128 * 4;
+  a.n_rb = (p->w + tsa::SC_ROWS - 1) / tsa::SC_ROWS;
+  a.scale_log2 = scale_of(p) * 1.4426950408889634f;
+  a.limit_ns = limit_ns_of(p);
+  const dim3 grid(a.n_chunks, bhq);
   const int rows = bhq * p->w;
+  if (cudaMemsetAsync(a.abort_word, 0, sizeof(uint32_t), st) != cudaSuccess) return TSA_ERR_CUDA;
   if (p->d == 128) {
-    if (!ensure_smem(g_st128, tsa::score_stats_kernel<128>, sm1) ||
-        !ensure_smem(g_sum128, tsa::score_sum_kernel<128>, sm2))
+    constexpr int sm = tsa::ScoreLayout<128>::ALLOC;
+    if (!ensure_smem(g_st128, tsa::score_kernel<128, false>, sm) ||
+        !ensure_smem(g_sum128, tsa::score_kernel<128, true>, sm))
       return TSA_ERR_CUDA;
-    tsa::score_stats_kernel<128><<<g1, tsa::SC_THREADS, sm1, st>>>(a);
+    tsa::score_kernel<128, false><<<grid, tsa::SC_THREADS, sm, st>>>(mq, mk, a);
     tsa::score_merge_kernel<<<(rows + 255) / 256, 256, 0, st>>>(a, rows);
-    tsa::score_sum_kernel<128><<<g2, tsa::SC_THREADS, sm2, st>>>(a);
+    tsa::score_kernel<128, true><<<grid, tsa::SC_THREADS, sm, st>>>(mq, mk, a);
   } else {
-    if (!ensure_smem(g_st64, tsa::score_stats_kernel<64>, sm1) ||
-        !ensure_smem(g_sum64, tsa::score_sum_kernel<64>, sm2))
+    constexpr int sm = tsa::ScoreLayout<64>::ALLOC;
+    if (!ensure_smem(g_st64, tsa::score_kernel<64, false>, sm) ||
+        !ensure_smem(g_sum64, tsa::score_kernel<64, true>, sm))
       return TSA_ERR_CUDA;
-    tsa::score_stats_kernel<64><<<g1, tsa::SC_THREADS, sm1, st>>>(a);
+    tsa::score_kernel<64, false><<<grid, tsa::SC_THREADS, sm, st>>>(mq, mk, a);
     tsa::score_merge_kernel<<<(rows + 255) / 256, 256, 0, st>>>(a, rows);
-    tsa::score_sum_kernel<64><<<g2, tsa::SC_THREADS, sm2, st>>>(a);
+    tsa::score_kernel<64, true><<<grid, tsa::SC_THREADS, sm, st>>>(mq, mk, a);
   }
   return launch_ok();
 }
@@ -290,7 +297,7 @@ bool tensors_ok(std::initializer_list<const void*> ptrs) {
 }
 
 uint32_t* status_of(void* ws) { return ws ? at<uint32_t>(ws, 0) : nullptr; }
-uint32_t* abort_of(void* ws) { return at<uint32_t>(ws, 4); }
+uint32_t* abort_of(void* ws) { return at<uint32_t>(ws, 4); }   // attention; +8: score
 
 }  // namespace
 
@@ -344,7 +351,7 @@ tsa_status tsa_stage_workspace_size(const tsa_params* p, size_t* bytes) {
 
 tsa_status tsa_reset_device_status(void* ws, void* stream) {
   if (!ws || !aligned(ws, kAlign)) return TSA_ERR_INVALID_ARG;
-  return cuda_ok(cudaMemsetAsync(ws, 0, 8, static_cast<cudaStream_t>(stream)));
+  return cuda_ok(cudaMemsetAsync(ws, 0, 16, static_cast<cudaStream_t>(stream)));
 }
 
 tsa_status tsa_get_device_status(const void* ws, void* stream, uint32_t* flags) {
