@@ -36,7 +36,7 @@ import workloads as W  # noqa: E402
 METRIC = "Token-sparse prefill attention ms and effective TFLOP/s at 128K vs dense; % BF16/HBM roofline"
 UNIT = "TFLOP/s (effective: dense causal attention FLOPs / TSA time)"
 DEFAULT_WORKLOAD = "c4_L128K_gqa"
-KERNELS_PER_FORWARD = 8  # score x3, budget, select, gather, attend, scatter
+KERNELS_PER_FORWARD = 8  # score x3, budget, select, gather, attention (scatter epilogue), zero fill
 
 
 def dense_flops(wl) -> float:
@@ -238,7 +238,8 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
     def forward():
         T.tsa_forward(p, q, k, v, o, ws, scores, idx, k_seq)
 
-    stage_names = ["score", "budget", "select", "gather", "attend", "scatter"]
+    # the kernels tsa_forward runs, one ABI call each
+    stage_names = ["score", "budget", "select", "gather", "attend"]
 
     def staged(evs):
         evs[0].record(stream)
@@ -250,10 +251,22 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
         evs[3].record(stream)
         T.tsa_gather_qkv(p, q, k, v, idx, k_seq, qc, kc, vc, ws)
         evs[4].record(stream)
-        T.tsa_attend(p, qc, kc, vc, k_seq, oc, None, ws)
+        T.tsa_attend_scatter(p, qc, kc, vc, idx, k_seq, o, None, ws)
         evs[5].record(stream)
+
+    # the separate stage calls the fused attention replaces (attention into a
+    # compressed output, then the scatter), and the fully fused gathering
+    # variant, timed for comparison and the scatter's own HBM roofline
+    unfused_names = ["attend_compressed", "scatter", "attend_gathered"]
+
+    def unfused(evs):
+        evs[0].record(stream)
+        T.tsa_attend(p, qc, kc, vc, k_seq, oc, None, ws)
+        evs[1].record(stream)
         T.tsa_scatter(p, oc, idx, k_seq, o, ws)
-        evs[6].record(stream)
+        evs[2].record(stream)
+        T.tsa_attend_gathered(p, q, k, v, idx, k_seq, o, None, ws)
+        evs[3].record(stream)
 
     def timed(fn, n):
         barrier()
@@ -278,16 +291,20 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
     ks = k_seq.cpu().numpy().tolist()
 
     # ---- per-stage breakdown (same kernels, one ABI call per stage)
-    per_stage = {n: [] for n in stage_names}
-    for it in range(args.warmup + args.steps):
-        evs = [torch.cuda.Event(enable_timing=True) for _ in range(7)]
-        barrier()
-        staged(evs)
-        torch.cuda.synchronize()
-        if it >= args.warmup:
-            for i, n in enumerate(stage_names):
-                per_stage[n].append(evs[i].elapsed_time(evs[i + 1]))
-    stage_ms = {n: rank_max(statistics.mean(v)) for n, v in per_stage.items()}
+    def breakdown(fn, names):
+        acc = {n: [] for n in names}
+        for it in range(args.warmup + args.steps):
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(names) + 1)]
+            barrier()
+            fn(evs)
+            torch.cuda.synchronize()
+            if it >= args.warmup:
+                for i, n in enumerate(names):
+                    acc[n].append(evs[i].elapsed_time(evs[i + 1]))
+        return {n: rank_max(statistics.mean(v)) for n, v in acc.items()}
+
+    stage_ms = breakdown(staged, stage_names)
+    unfused_ms = breakdown(unfused, unfused_names)
 
     # ---- dense baselines on the same tensors
     od = torch.empty_like(q)
@@ -327,7 +344,8 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
     cflops = compressed_flops(wl, ks)
     attn_ms = stage_ms["attend"]
     achieved = cflops / (attn_ms * 1e-3) / 1e12
-    roof = {"bound": "tensor", "kernel": "attend_kernel<128>", "achieved": achieved,
+    roof = {"bound": "tensor", "kernel": "attend2_kernel<128,2,false,true> (attention + scatter epilogue)",
+            "achieved": achieved,
             "peak": pk["bf16_sustained"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_sustained"],
             "traffic": None,
             "peak_note": f"bf16_tflops_sustained of {pk['source']} peaks (kernel timed inside a long step)"}
@@ -339,7 +357,8 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
         "scatter": tok * wl.d * 2 + kept * wl.d * 2,            # full write + kept rows read
         "score": 2 * wl.B * wl.Hkv * wl.L * wl.d * 2 + tok * 4,  # two K passes + scores
     }
-    stage_roof = {n: {"GB/s": b / (stage_ms[n] * 1e-3) / 1e9, "frac_hbm": b / (stage_ms[n] * 1e-3) / 1e9 / hbm}
+    times = {"gather": stage_ms["gather"], "scatter": unfused_ms["scatter"], "score": stage_ms["score"]}
+    stage_roof = {n: {"GB/s": b / (times[n] * 1e-3) / 1e9, "frac_hbm": b / (times[n] * 1e-3) / 1e9 / hbm}
                   for n, b in stage_bytes.items()}
 
     value = job_value(wl, world, ms)
@@ -359,7 +378,7 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
         "dense_ms": dense_ms, "speedup_vs_dense": dense_ms / ms, "sdpa_dense_ms": sdpa_ms,
         "effective_tflops": dense_flops(wl) / (ms * 1e-3) / 1e12,
         "achieved_tflops": cflops / (ms * 1e-3) / 1e12,
-        "stage_ms": stage_ms, "stage_hbm": stage_roof,
+        "stage_ms": stage_ms, "unfused_stage_ms": unfused_ms, "stage_hbm": stage_roof,
         "overhead_frac": (sum(stage_ms.values()) - attn_ms) / attn_ms,
         "roofline": roof, "cpu_baseline": cpu,
         "e2e": {"value": job_value(wl, world, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms,

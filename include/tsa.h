@@ -95,7 +95,9 @@ const char* tsa_status_string(tsa_status s);
 /* Host-only validation of p (the same checks every call makes). */
 tsa_status tsa_check_params(const tsa_params* p);
 
-/* Workspace bytes needed by tsa_forward (covers every stage call too). */
+/* Workspace bytes needed by tsa_forward (covers every stage call too): the
+ * stage scratch, scores, indices, budgets and the compressed Q, K and V (no
+ * compressed output is stored). */
 tsa_status tsa_workspace_size(const tsa_params* p, size_t* bytes);
 
 /* Workspace bytes needed by the single-stage calls below (status word and
@@ -138,6 +140,7 @@ tsa_status tsa_select(const tsa_params* p, const float* scores, const int32_t* k
 /* Step 4 -- gather.  [GS] "Arquitectura Central", compression:
  * qc[b,h,i] = q[b,h,S_h[i]], kc[b,h,i] = k[b,h/G,S_h[i]],
  * vc[b,h,i] = v[b,h/G,S_h[i]] for i < k_b.  Rows >= k_b are not written.
+ * qc may be NULL: then only K and V are gathered.
  * An index outside [0, L) writes a zero row and sets TSA_DEVFLAG_BAD_INDEX
  * (when ws is not NULL).  ws: NULL or stage size. */
 tsa_status tsa_gather_qkv(const tsa_params* p, const void* q, const void* k, const void* v,
@@ -155,6 +158,31 @@ tsa_status tsa_attend(const tsa_params* p, const void* qc, const void* kc, const
                       const int32_t* k_seq, void* oc, float* lse,
                       void* ws, size_t ws_bytes, void* stream);
 
+/* Steps 5-6 fused -- attention on the compressed tensors with the scatter in
+ * its epilogue.  [GS] "Arquitectura Central", decompression: compressed
+ * output row i is written straight to o[b,h,S_h[i]] and every other row of o
+ * is set to zero, so no compressed output is stored.  Same result as
+ * tsa_attend followed by tsa_scatter; this is what tsa_forward runs after
+ * tsa_gather_qkv.  In: qc, kc, vc (as tsa_attend), idx, k_seq.  Out: o
+ * [B,Hq,L,d]; lse (nullable) indexed by compressed row.  An index outside
+ * [0, L) is skipped and sets TSA_DEVFLAG_BAD_INDEX.  ws: stage size. */
+tsa_status tsa_attend_scatter(const tsa_params* p, const void* qc, const void* kc, const void* vc,
+                              const int32_t* idx, const int32_t* k_seq, void* o, float* lse,
+                              void* ws, size_t ws_bytes, void* stream);
+
+/* Steps 4-6 fused -- gather, compressed attention and scatter in one kernel.
+ * [GS] "Arquitectura Central": the same result as tsa_gather_qkv,
+ * tsa_attend and tsa_scatter in sequence, without materialising the
+ * compressed tensors: the attention kernel loads the rows S_h[i] of q and of
+ * k, v (KV head h/G) by index with TMA row gathers, and writes compressed
+ * output row i to o[b,h,S_h[i]]; every other row of o is set to zero.
+ * In: q, k, v (original layouts), idx, k_seq.  Out: o [B,Hq,L,d]; lse
+ * (nullable) indexed by compressed row as in tsa_attend.  An index outside
+ * [0, L) is skipped and sets TSA_DEVFLAG_BAD_INDEX.  ws: stage size. */
+tsa_status tsa_attend_gathered(const tsa_params* p, const void* q, const void* k, const void* v,
+                               const int32_t* idx, const int32_t* k_seq, void* o, float* lse,
+                               void* ws, size_t ws_bytes, void* stream);
+
 /* Dense causal GQA attention on the uncompressed tensors (the baseline the
  * method is measured against; the same kernel as tsa_attend with the
  * identity selection): o[b,h,i] = sum_{j<=i} softmax_j(scale *
@@ -168,10 +196,11 @@ tsa_status tsa_attend_dense(const tsa_params* p, const void* q, const void* k, c
 tsa_status tsa_scatter(const tsa_params* p, const void* oc, const int32_t* idx, const int32_t* k_seq,
                        void* o, void* ws, size_t ws_bytes, void* stream);
 
-/* The whole path: score -> budget -> select -> gather -> attend -> scatter,
- * enqueued on stream with no host synchronisation.  scores_out, idx_out,
- * k_seq_out may be NULL (then the workspace holds them); when given they
- * receive the intermediate results.  ws: >= tsa_workspace_size bytes. */
+/* The whole path: score -> budget -> select -> gather -> attention writing
+ * each output row in place, then zeros for the unselected rows (as
+ * tsa_attend_scatter); enqueued on stream with no host synchronisation.  scores_out, idx_out, k_seq_out may be NULL (then the
+ * workspace holds them); when given they receive the intermediate results.
+ * ws: >= tsa_workspace_size bytes. */
 tsa_status tsa_forward(const tsa_params* p, const void* q, const void* k, const void* v, void* o,
                        float* scores_out, int32_t* idx_out, int32_t* k_seq_out,
                        void* ws, size_t ws_bytes, void* stream);

@@ -76,8 +76,8 @@ def test_workspace_sizes(lib):
     p = good()
     full, stage = T.workspace_size(p), T.stage_workspace_size(p)
     assert stage < full
-    # forward holds at least scores, idx and four compressed tensors
-    assert full >= p.B * p.Hq * p.L * (4 + 4 + 4 * p.d * 2)
+    # forward holds scores, indices and compressed Q, K and V (never a compressed output)
+    assert p.B * p.Hq * p.L * (8 + 6 * p.d) <= full < p.B * p.Hq * p.L * (8 + 6 * p.d) + 2 * stage + 8192
     assert T.workspace_size(good(L=8192)) > full
     with pytest.raises(T.TSAError):
         T.workspace_size(good(d=96))
@@ -100,6 +100,8 @@ def test_null_and_misaligned_pointers_rejected(lib):
     assert _call(lib, "tsa_attend", p, FAKE, FAKE, FAKE, None, FAKE, None, FAKE, ws_n, None) == INVALID
     assert _call(lib, "tsa_attend_dense", p, FAKE, FAKE, None, FAKE, None, FAKE, ws_n, None) == INVALID
     assert _call(lib, "tsa_scatter", p, FAKE, FAKE, FAKE, None, None, 0, None) == INVALID
+    assert _call(lib, "tsa_attend_gathered", p, FAKE, FAKE, FAKE, None, FAKE, FAKE, None, FAKE, ws_n, None) == INVALID
+    assert _call(lib, "tsa_attend_gathered", p, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE, 64, None) == WORKSPACE
     assert _call(lib, "tsa_forward", p, FAKE, None, FAKE, FAKE, None, None, None, FAKE, big, None) == INVALID
     # misaligned tensors / workspace
     assert _call(lib, "tsa_score", p, odd, FAKE, FAKE, FAKE, ws_n, None) == INVALID

@@ -213,6 +213,93 @@ def test_attend_parity(name, tau):
     assert_status_clean(ws)
 
 
+@pytest.mark.parametrize("name", list(SHAPES))
+@pytest.mark.parametrize("tau", [0.05, 0.6])
+def test_attend_gathered_parity(name, tau):
+    """Gather, attention and scatter fused in one kernel (rows loaded by index,
+    outputs written in place, every other row zero) against the oracle."""
+    wl = SHAPES[name]
+    (q, k, v), (dq, dk, dv) = inputs(wl)
+    s32 = O.proxy_scores(q, k, wl.w)
+    _, k_seq = O.coverage_budget(s32, tau)
+    idx = O.select_topk(s32, k_seq)
+    p = P(wl, tau)
+    ws = T.new_workspace(p, full=False)
+    o = garbage_like(dq.shape)
+    lse = torch.full((wl.B, wl.Hq, wl.L), float("nan"), device="cuda")
+    T.tsa_attend_gathered(p, dq, dk, dv, dev_i32(idx), dev_i32(k_seq), o, lse, ws)
+    qc, kc, vc = O.gather_qkv(q, k, v, idx, k_seq)
+    oc = O.compressed_attention(qc, kc, vc, k_seq)
+    ref = O.scatter(oc, idx, k_seq, wl.L)
+    got = bf16_to_f64(o)
+    assert np.abs(got - ref).max() <= ATOL_OUT
+    bits = from_dev_bf16(o)
+    scale = O.default_scale(wl.d)
+    for b in range(wl.B):
+        kb = int(k_seq[b])
+        for h in range(wl.Hq):
+            unsel = np.setdiff1d(np.arange(wl.L), idx[b, h, :kb])
+            assert (bits[b, h, unsel] == 0).all()
+            i = kb - 1     # the last compressed row's log-sum-exp
+            x = (W.bf16_bits_to_f64(qc[b, h, i]) @ W.bf16_bits_to_f64(kc[b, h, :i + 1]).T) * scale
+            assert abs(float(lse[b, h, i]) - (x.max() + np.log(np.exp(x - x.max()).sum()))) < 1e-3
+    assert_status_clean(ws)
+
+
+@pytest.mark.parametrize("name", list(SHAPES))
+def test_attend_scatter_parity(name):
+    """The path tsa_forward runs: Q, K, V gathered once, then attention with
+    the scatter in its epilogue (outputs written in place, the rest zero)."""
+    wl = SHAPES[name]
+    (q, k, v), (dq, dk, dv) = inputs(wl)
+    s32 = O.proxy_scores(q, k, wl.w)
+    _, k_seq = O.coverage_budget(s32, wl.tau)
+    idx = O.select_topk(s32, k_seq)
+    p = P(wl)
+    ws = T.new_workspace(p, full=False)
+    shape = (wl.B, wl.Hq, wl.L, wl.d)
+    qc_d, kc, vc, o = (garbage_like(shape) for _ in range(4))
+    dix, dks = dev_i32(idx), dev_i32(k_seq)
+    T.tsa_gather_qkv(p, dq, dk, dv, dix, dks, None, kc, vc, ws)      # K/V-only form
+    T.tsa_gather_qkv(p, dq, dk, dv, dix, dks, qc_d, kc, vc, ws)
+    T.tsa_attend_scatter(p, qc_d, kc, vc, dix, dks, o, None, ws)
+    qc, kc_ref, vc_ref = O.gather_qkv(q, k, v, idx, k_seq)
+    for b in range(wl.B):      # the K/V-only gather is bit-exact
+        kb = int(k_seq[b])
+        assert np.array_equal(from_dev_bf16(kc)[b, :, :kb], kc_ref[b, :, :kb])
+        assert np.array_equal(from_dev_bf16(vc)[b, :, :kb], vc_ref[b, :, :kb])
+    ref = O.scatter(O.compressed_attention(qc, kc_ref, vc_ref, k_seq), idx, k_seq, wl.L)
+    assert np.abs(bf16_to_f64(o) - ref).max() <= ATOL_OUT
+    bits = from_dev_bf16(o)
+    for b in range(wl.B):
+        for h in range(wl.Hq):
+            unsel = np.setdiff1d(np.arange(wl.L), idx[b, h, :k_seq[b]])
+            assert (bits[b, h, unsel] == 0).all()
+    assert_status_clean(ws)
+
+
+def test_attend_gathered_flags_bad_index():
+    wl = SHAPES["gqa_d128_L1000"]
+    (q, k, v), (dq, dk, dv) = inputs(wl)
+    k_seq = np.array([300], dtype=np.int32)
+    idx = np.full((1, wl.Hq, wl.L), -1, dtype=np.int32)
+    for h in range(wl.Hq):
+        idx[0, h, :300] = np.arange(0, 900, 3)
+    idx[0, 1, 299] = wl.L + 5           # out of range: skipped and flagged, never written
+    p = P(wl)
+    ws = T.new_workspace(p, full=False)
+    o = garbage_like(dq.shape)
+    T.tsa_attend_gathered(p, dq, dk, dv, dev_i32(idx), dev_i32(k_seq), o, None, ws)
+    st, flags = T.get_device_status(ws)
+    assert flags & T.DEVFLAG_BAD_INDEX
+    qc, kc, vc = O.gather_qkv(q, k, v, np.where(idx >= 0, np.minimum(idx, wl.L - 1), -1), k_seq)
+    ref = O.compressed_attention(qc, kc, vc, k_seq)
+    got = bf16_to_f64(o)
+    for h in (0, 2, 3):                  # heads with valid indices are unaffected
+        assert np.abs(got[0, h, idx[0, h, :300]] - ref[0, h, :300]).max() <= ATOL_OUT
+    T.reset_device_status(ws)
+
+
 @pytest.mark.parametrize("name", ["c1_mha_d64_L1024", "gqa_d128_L1000", "gqa_d128_B2_L777_w130", "mha_d128_L129"])
 def test_attend_dense_parity(name):
     wl = SHAPES[name]

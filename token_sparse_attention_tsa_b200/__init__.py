@@ -28,7 +28,7 @@ DEVFLAG_NONFINITE, DEVFLAG_TIMEOUT, DEVFLAG_BAD_INDEX = 0x1, 0x2, 0x4
 EXPORTED = ("tsa_abi_version", "tsa_status_string", "tsa_check_params", "tsa_workspace_size",
             "tsa_stage_workspace_size", "tsa_reset_device_status", "tsa_get_device_status",
             "tsa_score", "tsa_budget", "tsa_select", "tsa_gather_qkv", "tsa_attend",
-            "tsa_attend_dense", "tsa_scatter", "tsa_forward", "tsa_score_noalloc")
+            "tsa_attend_dense", "tsa_attend_scatter", "tsa_attend_gathered", "tsa_scatter", "tsa_forward", "tsa_score_noalloc")
 
 
 class TSAError(RuntimeError):
@@ -80,6 +80,8 @@ def load(path: str | None = None):
             "tsa_gather_qkv": ([_P, _v, _v, _v, _v, _v, _v, _v, _v, _v, _sz, _v], ctypes.c_int),
             "tsa_attend": ([_P, _v, _v, _v, _v, _v, _v, _v, _sz, _v], ctypes.c_int),
             "tsa_attend_dense": ([_P, _v, _v, _v, _v, _v, _v, _sz, _v], ctypes.c_int),
+            "tsa_attend_gathered": ([_P, _v, _v, _v, _v, _v, _v, _v, _v, _sz, _v], ctypes.c_int),
+            "tsa_attend_scatter": ([_P, _v, _v, _v, _v, _v, _v, _v, _v, _sz, _v], ctypes.c_int),
             "tsa_scatter": ([_P, _v, _v, _v, _v, _v, _sz, _v], ctypes.c_int),
             "tsa_forward": ([_P, _v, _v, _v, _v, _v, _v, _v, _v, _sz, _v], ctypes.c_int),
             "tsa_score_noalloc": ([_P, _v, _v, _v, _v], ctypes.c_int),
@@ -208,7 +210,7 @@ def tsa_gather_qkv(p, q, k, v, idx, k_seq, qc, kc, vc, ws=None, stream=None):
     bf = torch.bfloat16
     _check(load().tsa_gather_qkv(ctypes.byref(p), _ptr(q, "q", bf), _ptr(k, "k", bf), _ptr(v, "v", bf),
                                  _ptr(idx, "idx", torch.int32), _ptr(k_seq, "k_seq", torch.int32),
-                                 _ptr(qc, "qc", bf), _ptr(kc, "kc", bf), _ptr(vc, "vc", bf),
+                                 _ptr(qc, "qc", bf), _ptr(kc, "kc", bf), _ptr(vc, "vc", bf),  # qc may be None
                                  _ptr(ws, "ws"), _nbytes(ws) if ws is not None else 0, _stream(stream)),
            "tsa_gather_qkv")
 
@@ -228,6 +230,24 @@ def tsa_attend_dense(p, q, k, v, o, lse, ws, stream=None):
     _check(load().tsa_attend_dense(ctypes.byref(p), _ptr(q, "q", bf), _ptr(k, "k", bf), _ptr(v, "v", bf),
                                    _ptr(o, "o", bf), _ptr(lse, "lse", torch.float32), _ptr(ws, "ws"),
                                    _nbytes(ws), _stream(stream)), "tsa_attend_dense")
+
+
+def tsa_attend_scatter(p, qc, kc, vc, idx, k_seq, o, lse, ws, stream=None):
+    import torch
+    bf = torch.bfloat16
+    _check(load().tsa_attend_scatter(ctypes.byref(p), _ptr(qc, "qc", bf), _ptr(kc, "kc", bf), _ptr(vc, "vc", bf),
+                                     _ptr(idx, "idx", torch.int32), _ptr(k_seq, "k_seq", torch.int32),
+                                     _ptr(o, "o", bf), _ptr(lse, "lse", torch.float32), _ptr(ws, "ws"),
+                                     _nbytes(ws), _stream(stream)), "tsa_attend_scatter")
+
+
+def tsa_attend_gathered(p, q, k, v, idx, k_seq, o, lse, ws, stream=None):
+    import torch
+    bf = torch.bfloat16
+    _check(load().tsa_attend_gathered(ctypes.byref(p), _ptr(q, "q", bf), _ptr(k, "k", bf), _ptr(v, "v", bf),
+                                      _ptr(idx, "idx", torch.int32), _ptr(k_seq, "k_seq", torch.int32),
+                                      _ptr(o, "o", bf), _ptr(lse, "lse", torch.float32), _ptr(ws, "ws"),
+                                      _nbytes(ws), _stream(stream)), "tsa_attend_gathered")
 
 
 def tsa_scatter(p, oc, idx, k_seq, o, ws=None, stream=None):

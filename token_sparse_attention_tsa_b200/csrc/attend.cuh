@@ -17,6 +17,8 @@
 
 #include <cuda_bf16.h>
 
+#include <type_traits>
+
 #include "sm100.cuh"
 
 namespace tsa {
@@ -27,6 +29,7 @@ struct AttnArgs {
   float* lse;             // [B*Hq, L] or null
   uint32_t* status;       // device status word or null
   uint32_t* abort_word;   // launch-wide abort word (zeroed before launch) or null
+  const int32_t* idx;     // gather mode: [B*Hq, L] selected rows (S_h ascending, then -1)
   int L;
   int Hq;
   int Hkv_map;            // heads of the K/V tensors
@@ -95,7 +98,14 @@ struct Attn2Layout {
   static constexpr int B_COUNT = B_DRAIN + 1;
 };
 
-template <int D, int PARTS>
+// kGather: Q, K and V rows are gathered by index (tile::gather4 from 2D maps
+// over [heads * L, d] with one-row boxes) instead of read as contiguous
+// compressed tiles.  (Each K/V tile is read by every later query tile of the
+// head, so gathering in the kernel repeats the gather many times; one gather
+// pass before the kernel is faster when compressed buffers can be held.)
+// kScatter: output row i is written to row idx[i] of o (in place in the
+// full-length output) instead of row i of a compressed output.
+template <int D, int PARTS, bool kGather, bool kScatter>
 __global__ void __launch_bounds__(Attn2Layout<D, PARTS>::THREADS, 1)
     attend2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
@@ -163,25 +173,47 @@ __global__ void __launch_bounds__(Attn2Layout<D, PARTS>::THREADS, 1)
         tma_prefetch_desc(&tmV);
       }
       const int zkv = b * a.Hkv_map + h / a.G_map;
-      if (leader) {
-        mbar_arrive_expect_tx(bar(C::B_Q), (two ? 2 : 1) * C::TILE);
+      // One 128-row tile into dst: a box load, or 32 four-row gathers whose
+      // row numbers come from idx (lane l reads entries 4l..4l+3; rows past
+      // the selection read row 0 of the head, masked or zeroed downstream).
+      auto load_tile = [&](auto by_index, uint32_t dst, const CUtensorMap* m, uint32_t br, int tile, int z) {
+        if constexpr (!decltype(by_index)::value) {
+          if (leader) {
 #pragma unroll
-        for (int c = 0; c < C::NCH; ++c) {
-          tma_load_3d(base + C::OFF_Q0 + c * C::CHUNK, &tmQ, bar(C::B_Q), c * 64, t0 * C::BM, bh);
-          if (two) tma_load_3d(base + C::OFF_Q1 + c * C::CHUNK, &tmQ, bar(C::B_Q), c * 64, (t0 + 1) * C::BM, bh);
+            for (int c = 0; c < C::NCH; ++c) tma_load_3d(dst + c * C::CHUNK, m, br, c * 64, tile * C::BM, z);
+          }
+        } else {
+          int rr[4];
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int i = tile * C::BM + 4 * lane + u;
+            const int v = i < valid ? __ldg(a.idx + static_cast<size_t>(bh) * a.L + i) : 0;
+            rr[u] = z * a.L + (v >= 0 && v < a.L ? v : 0);
+          }
+#pragma unroll 4
+          for (int g = 0; g < 32; ++g) {
+            const int r0 = __shfl_sync(0xffffffffu, rr[0], g), r1 = __shfl_sync(0xffffffffu, rr[1], g);
+            const int r2 = __shfl_sync(0xffffffffu, rr[2], g), r3 = __shfl_sync(0xffffffffu, rr[3], g);
+            if (leader) {
+#pragma unroll
+              for (int c = 0; c < C::NCH; ++c) tma_gather4(dst + c * C::CHUNK + g * 512, m, br, c * 64, r0, r1, r2, r3);
+            }
+          }
         }
-      }
+      };
+      if (leader) mbar_arrive_expect_tx(bar(C::B_Q), (two ? 2 : 1) * C::TILE);
+      __syncwarp();
+      constexpr std::integral_constant<bool, kGather> q_by_index{};
+      constexpr std::integral_constant<bool, kGather> kv_by_index{};
+      load_tile(q_by_index, base + C::OFF_Q0, &tmQ, bar(C::B_Q), t0, bh);
+      if (two) load_tile(q_by_index, base + C::OFF_Q1, &tmQ, bar(C::B_Q), t0 + 1, bh);
       int issued = 0;
       for (int n = 0; n < 2 * n_kv; ++n) {
         const int s = slot_of(n), u = use_of(n);
         if (u >= 1 && !__all_sync(0xffffffffu, mbar_wait(bar(C::B_EMPTY + s), (u - 1) & 1, wc))) break;
-        if (leader) {
-          mbar_arrive_expect_tx(bar(C::B_FULL + s), C::TILE);
-          const CUtensorMap* m = (n & 1) ? &tmV : &tmK;
-#pragma unroll
-          for (int c = 0; c < C::NCH; ++c)
-            tma_load_3d(ring(n) + c * C::CHUNK, m, bar(C::B_FULL + s), c * 64, (n >> 1) * C::BN, zkv);
-        }
+        if (leader) mbar_arrive_expect_tx(bar(C::B_FULL + s), C::TILE);
+        __syncwarp();
+        load_tile(kv_by_index, ring(n), (n & 1) ? &tmV : &tmK, bar(C::B_FULL + s), n >> 1, zkv);
         issued = n + 1;
       }
       if (leader && *cta_abort) {  // let every copy still in flight land before exit
@@ -418,13 +450,22 @@ __global__ void __launch_bounds__(Attn2Layout<D, PARTS>::THREADS, 1)
     if (live) {
       tc_fence_after();
       const float inv_l = 1.f / lt;
-      __nv_bfloat16* orow = a.o + (static_cast<size_t>(bh) * a.L + row) * D + half * (D / PARTS);
+      int orow_index = row;
+      bool store = row < valid;
+      if constexpr (kScatter) {  // compressed row i goes to token S_h[i]
+        orow_index = store ? __ldg(a.idx + static_cast<size_t>(bh) * a.L + row) : 0;
+        if (store && (orow_index < 0 || orow_index >= a.L)) {
+          store = false;
+          if (a.status) atomicOr(a.status, 0x4u);
+        }
+      }
+      __nv_bfloat16* orow = a.o + (static_cast<size_t>(bh) * a.L + (store ? orow_index : 0)) * D + half * (D / PARTS);
 #pragma unroll
       for (int c = 0; c < D / PARTS / 32; ++c) {
         float ov[32];
         tmem_ld32(o_col + c * 32, ov);
         tmem_ld_wait();
-        if (row < valid) {
+        if (store) {
           uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
 #pragma unroll
           for (int g = 0; g < 4; ++g) {

@@ -21,7 +21,7 @@ struct GatherArgs {
   const __nv_bfloat16 *q, *k, *v;  // [B*Hq, L, D], [B*Hkv, L, D] x2
   const int32_t* idx;              // [B*Hq, L]
   const int32_t* k_seq;            // [B]
-  __nv_bfloat16 *qc, *kc, *vc;     // [B*Hq, L, D]
+  __nv_bfloat16 *qc, *kc, *vc;     // [B*Hq, L, D]; qc may be null (K and V only)
   uint32_t* status;                // or null
   int L, Hq, Hkv, G;
   long long total_rows;            // B*Hq*L
@@ -46,17 +46,16 @@ __global__ void __launch_bounds__(256) gather_kernel(const GatherArgs a) {
     if (j < 0 || j >= a.L) {
       bad = true;
       const uint4 z = make_uint4(0, 0, 0, 0);
-      *reinterpret_cast<uint4*>(a.qc + dst) = z;
+      if (a.qc) *reinterpret_cast<uint4*>(a.qc + dst) = z;
       *reinterpret_cast<uint4*>(a.kc + dst) = z;
       *reinterpret_cast<uint4*>(a.vc + dst) = z;
       continue;
     }
     const size_t sq = (static_cast<size_t>(bh) * a.L + j) * D + sub * 8;
     const size_t skv = ((static_cast<size_t>(b) * a.Hkv + h / a.G) * a.L + j) * D + sub * 8;
-    const uint4 vq = __ldg(reinterpret_cast<const uint4*>(a.q + sq));
     const uint4 vk = __ldg(reinterpret_cast<const uint4*>(a.k + skv));
     const uint4 vv = __ldg(reinterpret_cast<const uint4*>(a.v + skv));
-    *reinterpret_cast<uint4*>(a.qc + dst) = vq;
+    if (a.qc) *reinterpret_cast<uint4*>(a.qc + dst) = __ldg(reinterpret_cast<const uint4*>(a.q + sq));
     *reinterpret_cast<uint4*>(a.kc + dst) = vk;
     *reinterpret_cast<uint4*>(a.vc + dst) = vv;
   }
@@ -77,7 +76,9 @@ constexpr int SCAT_ROWS = 256;  // output rows per CTA
 // grid (ceil(L/256), B*Hq), 256 threads.  The CTA maps its 256 output rows to
 // compressed positions through a shared table built from the ascending idx
 // (one binary search for the first entry), then writes every row once.
-template <int D>
+// kZeroOnly: write only the unselected rows (zeros) and leave the selected
+// ones, which the attention epilogue has already written in place.
+template <int D, bool kZeroOnly = false>
 __global__ void __launch_bounds__(256) scatter_kernel(const ScatterArgs a) {
   constexpr int LPR = D / 8;
   __shared__ int32_t where[SCAT_ROWS];
@@ -114,8 +115,10 @@ __global__ void __launch_bounds__(256) scatter_kernel(const ScatterArgs a) {
     const int r = r0 + rr;
     if (r >= a.L) break;
     const int i = where[rr];
+    if (kZeroOnly && i >= 0) continue;
     uint4 val = make_uint4(0, 0, 0, 0);
-    if (i >= 0) val = __ldg(reinterpret_cast<const uint4*>(a.oc + (static_cast<size_t>(bh) * a.L + i) * D + sub * 8));
+    if (!kZeroOnly && i >= 0)
+      val = __ldg(reinterpret_cast<const uint4*>(a.oc + (static_cast<size_t>(bh) * a.L + i) * D + sub * 8));
     __stcs(reinterpret_cast<uint4*>(a.o + (static_cast<size_t>(bh) * a.L + r) * D + sub * 8), val);
   }
   if (bad && a.status) atomicOr(a.status, 0x4u);

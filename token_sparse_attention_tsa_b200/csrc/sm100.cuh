@@ -305,3 +305,18 @@ __device__ __forceinline__ bool elect_one() {
 }
 
 }  // namespace tsa
+
+namespace tsa {
+
+// TMA row gather: rows r0..r3 (x columns from col) of a 2D tensor map whose
+// box is one row high land as four consecutive rows at dst.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* m, uint32_t bar, int col, int r0,
+                                            int r1, int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+      : "memory");
+}
+
+}  // namespace tsa

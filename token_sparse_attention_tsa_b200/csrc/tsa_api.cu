@@ -36,11 +36,13 @@ int score_chunks(const tsa_params* p) {
   return (p->L + span - 1) / span;
 }
 
-// Workspace layout.  Stage part: status word (+ abort word), score scratch.
-// Forward part: scores, idx, k_head, k_seq, qc, kc, vc, oc.
+// Workspace layout.  Stage part: status word (+ abort words), score scratch.
+// Forward part: scores, idx, k_head, k_seq and the compressed Q, K and V.
+// (tsa_forward's attention writes its output in place, so no compressed
+// output is stored.)
 struct WsLayout {
   size_t status = 0, part_m = 0, part_z = 0, stats = 0, stage_end = 0;
-  size_t scores = 0, idx = 0, k_head = 0, k_seq = 0, qc = 0, kc = 0, vc = 0, oc = 0, total = 0;
+  size_t scores = 0, idx = 0, k_head = 0, k_seq = 0, qc = 0, kc = 0, vc = 0, total = 0;
 };
 
 WsLayout layout_of(const tsa_params* p) {
@@ -55,15 +57,13 @@ WsLayout layout_of(const tsa_params* p) {
   w.stats = off;            off = align_up(off + rows * sizeof(float2));
   w.stage_end = off;
   const size_t tok = bhq * static_cast<size_t>(p->L);
-  const size_t ten = tok * static_cast<size_t>(p->d) * 2;
   w.scores = off;           off = align_up(off + tok * sizeof(float));
   w.idx = off;              off = align_up(off + tok * sizeof(int32_t));
   w.k_head = off;           off = align_up(off + bhq * sizeof(int32_t));
   w.k_seq = off;            off = align_up(off + static_cast<size_t>(p->B) * sizeof(int32_t));
-  w.qc = off;               off = align_up(off + ten);
-  w.kc = off;               off = align_up(off + ten);
-  w.vc = off;               off = align_up(off + ten);
-  w.oc = off;               off = align_up(off + ten);
+  w.qc = off;               off = align_up(off + tok * static_cast<size_t>(p->d) * 2);
+  w.kc = off;               off = align_up(off + tok * static_cast<size_t>(p->d) * 2);
+  w.vc = off;               off = align_up(off + tok * static_cast<size_t>(p->d) * 2);
   w.total = off;
   return w;
 }
@@ -114,6 +114,20 @@ bool make_map(CUtensorMap* m, const void* base, int d, int L, int heads, int box
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [rows, d] bf16 viewed as one 2D tensor; box = one row x 64 columns,
+// 128-byte swizzle (the form tile::gather4 loads need).
+bool make_row_map(CUtensorMap* m, const void* base, int d, long long rows) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * 2};
+  cuuint32_t box[2] = {64, 1};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // ---------------------------------------------------------------- attributes
 template <typename K>
 bool ensure_smem(std::atomic<int> (&done)[kMaxDevices], K kernel, int bytes) {
@@ -126,7 +140,8 @@ bool ensure_smem(std::atomic<int> (&done)[kMaxDevices], K kernel, int bytes) {
   return true;
 }
 
-std::atomic<int> g_attn64[kMaxDevices], g_attn128[kMaxDevices], g_st64[kMaxDevices],
+std::atomic<int> g_attn64[kMaxDevices], g_attn128[kMaxDevices], g_gath64[kMaxDevices], g_gath128[kMaxDevices],
+    g_gq64[kMaxDevices], g_gq128[kMaxDevices], g_st64[kMaxDevices],
     g_st128[kMaxDevices], g_sum64[kMaxDevices], g_sum128[kMaxDevices], g_budget[kMaxDevices],
     g_select[kMaxDevices];
 
@@ -245,16 +260,29 @@ tsa_status run_scatter(const tsa_params* p, const void* oc, const int32_t* idx, 
 }
 
 // Attention over [B*Hq, L, d] queries against K/V with heads_kv heads
+// (query head h of sequence b reads K/V head b*heads_kv + h/g_kv).  With idx,
+// Q/K/V rows are gathered by index inside the kernel and output row i lands
+// at row idx[i] of o (the rest of o is not touched).
+// Attention over [B*Hq, L, d] queries against K/V with heads_kv heads
 // (query head h of sequence b reads K/V head b*heads_kv + h/g_kv).
+// idx (with scatter): output row i lands at row idx[i] of o (the rest of o is
+// not touched).  idx with gather as well: Q/K/V rows are loaded by index from
+// the uncompressed tensors instead of as compressed tiles.
 tsa_status run_attend(const tsa_params* p, const void* q, const void* k, const void* v, int heads_kv, int g_kv,
                       const int32_t* k_seq, void* o, float* lse, uint32_t* status, uint32_t* abort_word,
-                      cudaStream_t st) {
+                      cudaStream_t st, const int32_t* idx = nullptr, bool gather = false) {
   CUtensorMap mq, mk, mv;
   const int bhq = p->B * p->Hq;
   const int bhkv = p->B * heads_kv;
-  if (!make_map(&mq, q, p->d, p->L, bhq) || !make_map(&mk, k, p->d, p->L, bhkv) ||
-      !make_map(&mv, v, p->d, p->L, bhkv))
-    return TSA_ERR_CUDA;
+  const bool scatter = idx != nullptr;
+  gather = gather && scatter;
+  const bool maps_ok =
+      gather ? (make_row_map(&mq, q, p->d, static_cast<long long>(bhq) * p->L) &&
+                make_row_map(&mk, k, p->d, static_cast<long long>(bhkv) * p->L) &&
+                make_row_map(&mv, v, p->d, static_cast<long long>(bhkv) * p->L))
+             : (make_map(&mq, q, p->d, p->L, bhq) && make_map(&mk, k, p->d, p->L, bhkv) &&
+                make_map(&mv, v, p->d, p->L, bhkv));
+  if (!maps_ok) return TSA_ERR_CUDA;
   if (cudaMemsetAsync(abort_word, 0, sizeof(uint32_t), st) != cudaSuccess) return TSA_ERR_CUDA;
   tsa::AttnArgs a;
   a.k_seq = k_seq;
@@ -262,6 +290,7 @@ tsa_status run_attend(const tsa_params* p, const void* q, const void* k, const v
   a.lse = lse;
   a.status = status;
   a.abort_word = abort_word;
+  a.idx = idx;
   a.L = p->L;
   a.Hq = p->Hq;
   a.Hkv_map = heads_kv;
@@ -270,15 +299,34 @@ tsa_status run_attend(const tsa_params* p, const void* q, const void* k, const v
   a.scale_log2 = scale_of(p) * 1.4426950408889634f;
   a.limit_ns = limit_ns_of(p);
   const dim3 grid((a.n_tiles + 1) / 2, bhq);  // two query tiles per CTA
+  auto launch = [&](auto kernel, std::atomic<int>(&attr)[kMaxDevices], int threads, int smem) -> tsa_status {
+    if (!ensure_smem(attr, kernel, smem)) return TSA_ERR_CUDA;
+    kernel<<<grid, threads, smem, st>>>(mq, mk, mv, a);
+    return launch_ok();
+  };
+  constexpr int P = kSoftmaxParts;
   if (p->d == 128) {
-    using L = tsa::Attn2Layout<128, kSoftmaxParts>;
-    if (!ensure_smem(g_attn128, tsa::attend2_kernel<128, kSoftmaxParts>, L::ALLOC)) return TSA_ERR_CUDA;
-    tsa::attend2_kernel<128, kSoftmaxParts><<<grid, L::THREADS, L::ALLOC, st>>>(mq, mk, mv, a);
-  } else {
-    using L = tsa::Attn2Layout<64, kSoftmaxParts>;
-    if (!ensure_smem(g_attn64, tsa::attend2_kernel<64, kSoftmaxParts>, L::ALLOC)) return TSA_ERR_CUDA;
-    tsa::attend2_kernel<64, kSoftmaxParts><<<grid, L::THREADS, L::ALLOC, st>>>(mq, mk, mv, a);
+    using L = tsa::Attn2Layout<128, P>;
+    if (!scatter) return launch(tsa::attend2_kernel<128, P, false, false>, g_attn128, L::THREADS, L::ALLOC);
+    if (!gather) return launch(tsa::attend2_kernel<128, P, false, true>, g_gq128, L::THREADS, L::ALLOC);
+    return launch(tsa::attend2_kernel<128, P, true, true>, g_gath128, L::THREADS, L::ALLOC);
   }
+  using L = tsa::Attn2Layout<64, P>;
+  if (!scatter) return launch(tsa::attend2_kernel<64, P, false, false>, g_attn64, L::THREADS, L::ALLOC);
+  if (!gather) return launch(tsa::attend2_kernel<64, P, false, true>, g_gq64, L::THREADS, L::ALLOC);
+  return launch(tsa::attend2_kernel<64, P, true, true>, g_gath64, L::THREADS, L::ALLOC);
+}
+
+// Zero the rows of o that no index selects (the selected rows are left as
+// they are).
+tsa_status run_zero_unselected(const tsa_params* p, const int32_t* idx, const int32_t* k_seq, void* o,
+                               uint32_t* status, cudaStream_t st) {
+  tsa::ScatterArgs a{nullptr, idx, k_seq, static_cast<__nv_bfloat16*>(o), status, p->L, p->Hq};
+  const dim3 g((p->L + tsa::SCAT_ROWS - 1) / tsa::SCAT_ROWS, p->B * p->Hq);
+  if (p->d == 128)
+    tsa::scatter_kernel<128, true><<<g, 256, 0, st>>>(a);
+  else
+    tsa::scatter_kernel<64, true><<<g, 256, 0, st>>>(a);
   return launch_ok();
 }
 
@@ -399,7 +447,7 @@ tsa_status tsa_gather_qkv(const tsa_params* p, const void* q, const void* k, con
                           void* stream) {
   tsa_status s = tsa_check_params(p);
   if (s != TSA_OK) return s;
-  if (!tensors_ok({q, k, v, idx, k_seq, qc, kc, vc})) return TSA_ERR_INVALID_ARG;
+  if (!tensors_ok({q, k, v, idx, k_seq, kc, vc}) || (qc && !aligned(qc, 16))) return TSA_ERR_INVALID_ARG;
   if (ws && (s = check_ws(p, ws, ws_bytes, false)) != TSA_OK) return s;
   return run_gather(p, q, k, v, idx, k_seq, qc, kc, vc, status_of(ws), static_cast<cudaStream_t>(stream));
 }
@@ -448,17 +496,45 @@ tsa_status tsa_forward(const tsa_params* p, const void* q, const void* k, const 
   float* scores = scores_out ? scores_out : at<float>(ws, w.scores);
   int32_t* idx = idx_out ? idx_out : at<int32_t>(ws, w.idx);
   int32_t* kseq = k_seq_out ? k_seq_out : at<int32_t>(ws, w.k_seq);
-  void* qc = at<void>(ws, w.qc);
-  void* kc = at<void>(ws, w.kc);
-  void* vc = at<void>(ws, w.vc);
-  void* oc = at<void>(ws, w.oc);
   if ((s = run_score(p, q, k, scores, ws, st)) != TSA_OK) return s;
   if ((s = run_budget(p, scores, at<int32_t>(ws, w.k_head), kseq, status_of(ws), st)) != TSA_OK) return s;
   if ((s = run_select(p, scores, kseq, idx, st)) != TSA_OK) return s;
+  // gather once, attention writing each output row in place, zeros for the
+  // unselected rows (tsa_gather_qkv + tsa_attend_scatter)
+  void* qc = at<void>(ws, w.qc);
+  void* kc = at<void>(ws, w.kc);
+  void* vc = at<void>(ws, w.vc);
   if ((s = run_gather(p, q, k, v, idx, kseq, qc, kc, vc, status_of(ws), st)) != TSA_OK) return s;
-  if ((s = run_attend(p, qc, kc, vc, p->Hq, 1, kseq, oc, nullptr, status_of(ws), abort_of(ws), st)) != TSA_OK)
+  if ((s = run_attend(p, qc, kc, vc, p->Hq, 1, kseq, o, nullptr, status_of(ws), abort_of(ws), st, idx)) != TSA_OK)
     return s;
-  return run_scatter(p, oc, idx, kseq, o, status_of(ws), st);
+  return run_zero_unselected(p, idx, kseq, o, status_of(ws), st);
+}
+
+tsa_status tsa_attend_scatter(const tsa_params* p, const void* qc, const void* kc, const void* vc,
+                              const int32_t* idx, const int32_t* k_seq, void* o, float* lse, void* ws,
+                              size_t ws_bytes, void* stream) {
+  tsa_status s = tsa_check_params(p);
+  if (s != TSA_OK) return s;
+  if (!tensors_ok({qc, kc, vc, idx, k_seq, o}) || (lse && !aligned(lse, 4))) return TSA_ERR_INVALID_ARG;
+  if ((s = check_ws(p, ws, ws_bytes, false)) != TSA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = run_attend(p, qc, kc, vc, p->Hq, 1, k_seq, o, lse, status_of(ws), abort_of(ws), st, idx)) != TSA_OK)
+    return s;
+  return run_zero_unselected(p, idx, k_seq, o, status_of(ws), st);
+}
+
+tsa_status tsa_attend_gathered(const tsa_params* p, const void* q, const void* k, const void* v,
+                               const int32_t* idx, const int32_t* k_seq, void* o, float* lse, void* ws,
+                               size_t ws_bytes, void* stream) {
+  tsa_status s = tsa_check_params(p);
+  if (s != TSA_OK) return s;
+  if (!tensors_ok({q, k, v, idx, k_seq, o}) || (lse && !aligned(lse, 4))) return TSA_ERR_INVALID_ARG;
+  if ((s = check_ws(p, ws, ws_bytes, false)) != TSA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = run_attend(p, q, k, v, p->Hkv, p->Hq / p->Hkv, k_seq, o, lse, status_of(ws), abort_of(ws), st, idx,
+                      true)) != TSA_OK)
+    return s;
+  return run_zero_unselected(p, idx, k_seq, o, status_of(ws), st);
 }
 
 }  // extern "C"
