@@ -37,6 +37,11 @@ METRIC = "Token-sparse prefill attention ms and effective TFLOP/s at 128K vs den
 UNIT = "TFLOP/s (effective: dense causal attention FLOPs / TSA time)"
 DEFAULT_WORKLOAD = "c4_L128K_gqa"
 KERNELS_PER_FORWARD = 8  # score x3, budget, select, gather, attention (scatter epilogue), zero fill
+# DRAM bytes per kept (head, row) of the attention kernel with the scatter
+# epilogue, from ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch
+# on the 32K workload (812.6 MB for 32 x 25147 kept rows); DRAM traffic grows
+# with kept rows, not with FLOPs (algorithmic: 3 x 256 B read + 256 B written).
+ATTN_DRAM_BYTES_PER_KEPT_ROW = 812.6e6 / (32 * 25147)
 
 
 def dense_flops(wl) -> float:
@@ -347,7 +352,8 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
     roof = {"bound": "tensor", "kernel": "attend2_kernel<128,2,false,true> (attention + scatter epilogue)",
             "achieved": achieved,
             "peak": pk["bf16_sustained"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_sustained"],
-            "traffic": None,
+            "traffic": ATTN_DRAM_BYTES_PER_KEPT_ROW * wl.Hq * sum(ks),
+            "traffic_note": "ncu DRAM bytes of one launch on the 32K workload, scaled by kept rows",
             "peak_note": f"bf16_tflops_sustained of {pk['source']} peaks (kernel timed inside a long step)"}
     hbm = pk["hbm_gbs"]
     tok = wl.B * wl.Hq * wl.L
