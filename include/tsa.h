@@ -72,6 +72,13 @@ typedef enum tsa_status {
   TSA_ERR_BAD_INDEX = 7     /* device status: an index was outside [0, L)    */
 } tsa_status;
 
+/* tsa_params.flags: test hook for the failure path.  The attention kernels
+ * (tsa_attend*, tsa_forward) first wait on a barrier that nothing completes;
+ * the bounded wait runs out after timeout_ms, the kernel sets
+ * TSA_DEVFLAG_TIMEOUT, lets its in-flight copies land, frees its tensor
+ * memory and returns without writing outputs.  The context stays usable. */
+#define TSA_FLAG_TEST_STALL 0x80000000u
+
 /* Bits of the device status word (first 4 bytes of ws). */
 #define TSA_DEVFLAG_NONFINITE 0x1u
 #define TSA_DEVFLAG_TIMEOUT 0x2u
@@ -82,7 +89,7 @@ typedef struct tsa_params {
   int32_t w;            /* proxy window: the last w query positions          */
   float tau;            /* coverage threshold, 0 <= tau < 1                  */
   float softmax_scale;  /* 0 selects 1/sqrt(d) (fp32)                        */
-  uint32_t flags;       /* reserved, must be 0                               */
+  uint32_t flags;       /* 0, or TSA_FLAG_TEST_STALL (failure-path test)     */
   uint32_t timeout_ms;  /* limit of one pipeline wait; 0 selects 2000 ms     */
 } tsa_params;
 

@@ -66,10 +66,12 @@ def test_param_validation(lib, kw, want):
     assert T.check_params(p) == want
 
 
-def test_flags_must_be_zero(lib):
+def test_flags_only_the_test_hook(lib):
     p = good()
     p.flags = 1
     assert T.check_params(p) == INVALID
+    p.flags = T.FLAG_TEST_STALL
+    assert T.check_params(p) == 0
 
 
 def test_workspace_sizes(lib):

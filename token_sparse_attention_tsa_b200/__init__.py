@@ -23,6 +23,7 @@ TSA_OK = 0
 STATUS_NAMES = {0: "TSA_OK", 1: "TSA_ERR_INVALID_ARG", 2: "TSA_ERR_UNSUPPORTED", 3: "TSA_ERR_WORKSPACE",
                 4: "TSA_ERR_CUDA", 5: "TSA_ERR_NONFINITE", 6: "TSA_ERR_TIMEOUT", 7: "TSA_ERR_BAD_INDEX"}
 DEVFLAG_NONFINITE, DEVFLAG_TIMEOUT, DEVFLAG_BAD_INDEX = 0x1, 0x2, 0x4
+FLAG_TEST_STALL = 0x80000000
 
 # Every symbol the header declares (checked by the tests).
 EXPORTED = ("tsa_abi_version", "tsa_status_string", "tsa_check_params", "tsa_workspace_size",
@@ -44,8 +45,8 @@ class tsa_params(ctypes.Structure):
                 ("flags", ctypes.c_uint32), ("timeout_ms", ctypes.c_uint32)]
 
 
-def params(B, Hq, Hkv, L, d, w, tau, softmax_scale=0.0, timeout_ms=0) -> tsa_params:
-    return tsa_params(B, Hq, Hkv, L, d, w, tau, softmax_scale, 0, timeout_ms)
+def params(B, Hq, Hkv, L, d, w, tau, softmax_scale=0.0, timeout_ms=0, flags=0) -> tsa_params:
+    return tsa_params(B, Hq, Hkv, L, d, w, tau, softmax_scale, flags, timeout_ms)
 
 
 _lock = threading.Lock()

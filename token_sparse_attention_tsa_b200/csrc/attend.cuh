@@ -37,6 +37,7 @@ struct AttnArgs {
   int n_tiles;            // ceil(L / 128)
   float scale_log2;       // softmax scale * log2(e)
   uint64_t limit_ns;      // per-wait time limit
+  int test_stall;         // failure-path test: the MMA issuer first waits on a barrier nothing completes
 };
 
 // ---------------------------------------------------------------------------
@@ -270,7 +271,9 @@ __global__ void __launch_bounds__(Attn2Layout<D, PARTS>::THREADS, 1)
         return __all_sync(0xffffffffu, mbar_wait(br, par, wc));
       };
       auto full = [&](int n) { return wait_all(bar(C::B_FULL + slot_of(n)), use_of(n) & 1); };
-      bool ok = wait_all(bar(C::B_Q), 0);
+      // test hook: phase 0 of the drain barrier completes only at teardown,
+      // so this bounded wait runs out and takes the abort path
+      bool ok = !(a.test_stall && !wait_all(bar(C::B_DRAIN), 0)) && wait_all(bar(C::B_Q), 0);
       for (int j = 0; ok && j < n_kv; ++j) {
         if (!(ok = full(2 * j))) break;                                  // K_j
         tc_fence_after();

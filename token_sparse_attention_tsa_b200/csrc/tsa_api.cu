@@ -298,6 +298,7 @@ tsa_status run_attend(const tsa_params* p, const void* q, const void* k, const v
   a.n_tiles = (p->L + 127) / 128;
   a.scale_log2 = scale_of(p) * 1.4426950408889634f;
   a.limit_ns = limit_ns_of(p);
+  a.test_stall = (p->flags & TSA_FLAG_TEST_STALL) ? 1 : 0;
   const dim3 grid((a.n_tiles + 1) / 2, bhq);  // two query tiles per CTA
   auto launch = [&](auto kernel, std::atomic<int>(&attr)[kMaxDevices], int threads, int smem) -> tsa_status {
     if (!ensure_smem(attr, kernel, smem)) return TSA_ERR_CUDA;
@@ -374,7 +375,7 @@ tsa_status tsa_check_params(const tsa_params* p) {
   if (p->w > p->L) return TSA_ERR_INVALID_ARG;
   if (!(p->tau >= 0.f && p->tau < 1.f)) return TSA_ERR_INVALID_ARG;
   if (!(p->softmax_scale >= 0.f) || std::isinf(p->softmax_scale)) return TSA_ERR_INVALID_ARG;
-  if (p->flags != 0) return TSA_ERR_INVALID_ARG;
+  if ((p->flags & ~TSA_FLAG_TEST_STALL) != 0) return TSA_ERR_INVALID_ARG;
   if (p->d != 64 && p->d != 128) return TSA_ERR_UNSUPPORTED;
   if (p->w > 4096 || p->L > (1 << 22)) return TSA_ERR_UNSUPPORTED;
   if (static_cast<long long>(p->B) * p->Hq * p->L >= (1LL << 31)) return TSA_ERR_UNSUPPORTED;
