@@ -344,16 +344,14 @@ __global__ void __launch_bounds__(Attn2Layout<D, PARTS>::THREADS, 1)
             for (int e = 0; e < 32; ++e)
               if ((half * C::COLS + c * 32 + e) > r) sv[c][e] = -INFINITY;
         }
-        float m8[8];
+        // row max: four chains of three-input maxima over value pairs
+        float m4[4] = {sv[0][0], sv[0][1], sv[0][2], sv[0][3]};
 #pragma unroll
-        for (int u = 0; u < 8; ++u) m8[u] = sv[0][u];
-#pragma unroll
-        for (int c = 0; c < NC; ++c)
-#pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (c > 0 || e >= 8) m8[e & 7] = fmaxf(m8[e & 7], sv[c][e]);
-        mh = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
-                   fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+        for (int i = 4; i < C::COLS; i += 2) {       // i even: i, i+1 lie in one 32-chunk
+          const int u = (i >> 1) & 3;
+          m4[u] = fmax3(m4[u], sv[i >> 5][i & 31], sv[i >> 5][(i & 31) + 1]);
+        }
+        mh = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
       }
       float mx = mh;
       if constexpr (PARTS == 2) {
@@ -369,9 +367,10 @@ __global__ void __launch_bounds__(Attn2Layout<D, PARTS>::THREADS, 1)
       const float alpha = resc ? ex2_approx(m_used - m_new) : 1.f;
       if (resc) m_used = m_new;
       const float nm = -m_used;
-      float r8[8];
+      const uint64_t sl2x2 = f2_pack(sl2, sl2), nmx2 = f2_pack(nm, nm);
+      uint64_t r4[4];                               // packed partial row sums
 #pragma unroll
-      for (int u = 0; u < 8; ++u) r8[u] = 0.f;
+      for (int u = 0; u < 4; ++u) r4[u] = 0ull;
       // pass 2: S columns [32c, 32c+32) of the part give P columns
       // [16c, 16c+16), which lie in columns already read.
 #pragma unroll
@@ -387,14 +386,19 @@ __global__ void __launch_bounds__(Attn2Layout<D, PARTS>::THREADS, 1)
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float p0 = ex2_approx(fmaf(sv[2 * e], sl2, nm));
-          const float p1 = ex2_approx(fmaf(sv[2 * e + 1], sl2, nm));
-          r8[e & 7] += p0 + p1;
+          float x0, x1;
+          f2_unpack(f2_fma(f2_pack(sv[2 * e], sv[2 * e + 1]), sl2x2, nmx2), x0, x1);
+          const float p0 = ex2_approx(x0);
+          const float p1 = ex2_approx(x1);
+          r4[e & 3] = f2_add(r4[e & 3], f2_pack(p0, p1));
           pk[e] = pack_bf16x2(p0, p1);
         }
         tmem_st16u(p_col + c * 16, pk);
       }
-      l = l * alpha + (((r8[0] + r8[1]) + (r8[2] + r8[3])) + ((r8[4] + r8[5]) + (r8[6] + r8[7])));
+      float rs[8];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) f2_unpack(r4[u], rs[2 * u], rs[2 * u + 1]);
+      l = l * alpha + (((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7])));
       // O is rescaled only when a row's max grew past the lazy threshold, and
       // then only once the previous P.V into O has completed (and before this
       // tile's P.V, which waits for P_FULL).  Otherwise the wait is skipped:
