@@ -42,22 +42,24 @@ struct AttnArgs {
 
 // ---------------------------------------------------------------------------
 // Two query tiles per CTA (rows [256c, 256c+256) of one head), ping-ponged,
-// with two softmax warpgroups per tile:
-//   warps 0..7   softmax of query tile 0 (warps 0..3 columns 0..63 of every
-//                row, warps 4..7 columns 64..127)
-//   warps 8..15  softmax of query tile 1 (same split)
-//   warp 16      TMEM allocator + MMA issuer
-//   warp 17      TMA producer
-// Each row's max and sum are combined across its two halves through shared
-// memory behind a named barrier of the tile's 256 threads; the barrier also
+// with PARTS softmax warpgroups per tile (each row's 128 S columns split in
+// PARTS parts):
+//   warps 0..4*PARTS-1          softmax of query tile 0 (warp w: rows
+//                               32(w%4)..+32, part w/4)
+//   warps 4*PARTS..8*PARTS-1    softmax of query tile 1 (same split)
+//   warp 8*PARTS                TMEM allocator + MMA issuer
+//   warp 8*PARTS+1              TMA producer
+// PARTS = 1 is the configuration in use: one thread owns a whole row, holds
+// its 128 S values in registers between the max and the exponentials, and
+// needs no exchange.  With PARTS = 2 (18 warps, so at most 96 registers a
+// thread) each row's max and sum are combined across its two halves through
+// shared memory behind a named barrier of the tile's 256 threads that also
 // ANDs the threads' progress flags, so both halves always take the same
-// branch (a timed-out wait can never leave one half at a barrier alone).
+// branch, and S is re-read from TMEM for the exponentials.
 // TMEM: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D, 256+2D).  Each
-// half writes its 64 P values (bf16, two per 32-bit column) over the first 32
-// of its own 64 S columns, and the P.V MMA reads P from TMEM (k-steps 0..3
-// from the first half's columns, 4..7 from the second's), so P never touches
-// shared memory.  The softmax reads S twice (row max first, then the
-// exponentials), keeping only 32 values in registers at a time.  K and V
+// part writes its P values (bf16, two per 32-bit column) over the first half
+// of its own S columns, and the P.V MMA reads P from TMEM, so P never touches
+// shared memory.  K and V
 // tiles stream through one TMA ring of NSLOT slots in the order K0 V0 K1 V1 ...
 // Per KV tile j the MMA warp issues S0_j, PV1_{j-1}, S1_j, PV0_j: while one
 // tile's softmax runs the tensor core works on the other tile.  S0_{j+1}
@@ -273,10 +275,14 @@ __global__ void __launch_bounds__(Attn2Layout<D, PARTS>::THREADS, 1)
       auto full = [&](int n) { return wait_all(bar(C::B_FULL + slot_of(n)), use_of(n) & 1); };
       // test hook: phase 0 of the drain barrier completes only at teardown,
       // so this bounded wait runs out and takes the abort path
-      bool ok = !(a.test_stall && !wait_all(bar(C::B_DRAIN), 0)) && wait_all(bar(C::B_Q), 0);
+      // The waits for K_{j+1} and V_j come before the wait for P0_j: those
+      // tiles have normally landed long before, and once P0_j arrives PV0_j
+      // and S0_{j+1} go out back to back.  Every slot these loads need was
+      // released by a commit issued earlier in this loop, so waiting for them
+      // here cannot deadlock the ring.
+      bool ok = !(a.test_stall && !wait_all(bar(C::B_DRAIN), 0)) && wait_all(bar(C::B_Q), 0) && full(0);
       for (int j = 0; ok && j < n_kv; ++j) {
-        if (!(ok = full(2 * j))) break;                                  // K_j
-        tc_fence_after();
+        tc_fence_after();                                                // K_j has landed
         if (j <= last0) issue_s(0, j);
         if (two && j >= 1) {
           if (!(ok = wait_all(bar(C::B_P + 1), (j - 1) & 1))) break;
@@ -286,12 +292,16 @@ __global__ void __launch_bounds__(Attn2Layout<D, PARTS>::THREADS, 1)
         }
         if (two) issue_s(1, j);
         commit_to(bar(C::B_EMPTY + slot_of(2 * j)));                     // K_j done
+        const bool more = j + 1 < n_kv;
         if (j <= last0) {
-          if (!(ok = wait_all(bar(C::B_P + 0), j & 1))) break;
           if (!(ok = full(2 * j + 1))) break;                            // V_j
+          if (more && !(ok = full(2 * j + 2))) break;                    // K_{j+1}
+          if (!(ok = wait_all(bar(C::B_P + 0), j & 1))) break;
           tc_fence_after();
           issue_pv(0, j);
           if (!two) commit_to(bar(C::B_EMPTY + slot_of(2 * j + 1)));
+        } else if (more && !(ok = full(2 * j + 2))) {
+          break;
         }
       }
       if (ok && two) {
@@ -330,10 +340,10 @@ __global__ void __launch_bounds__(Attn2Layout<D, PARTS>::THREADS, 1)
       live = live && __all_sync(0xffffffffu, mbar_wait(bar(C::B_S + tt), j & 1, wc));
       float mh = -INFINITY;
       const bool diag = (j == last);
+      constexpr int NC = C::COLS / 32;
+      float sv[NC][32];
       if (live) {  // pass 1: this part's row max
         tc_fence_after();
-        constexpr int NC = C::COLS / 32;
-        float sv[NC][32];
 #pragma unroll
         for (int c = 0; c < NC; ++c) tmem_ld32(s_col + c * 32, sv[c]);
         tmem_ld_wait();
@@ -372,22 +382,26 @@ __global__ void __launch_bounds__(Attn2Layout<D, PARTS>::THREADS, 1)
 #pragma unroll
       for (int u = 0; u < 4; ++u) r4[u] = 0ull;
       // pass 2: S columns [32c, 32c+32) of the part give P columns
-      // [16c, 16c+16), which lie in columns already read.
+      // [16c, 16c+16), which lie in columns already read.  A thread that
+      // owns a whole row still holds its S values from pass 1; with the row
+      // split in parts the register budget only allows re-reading them.
 #pragma unroll
-      for (int c = 0; c < C::COLS / 32; ++c) {
-        float sv[32];
-        tmem_ld32(s_col + c * 32, sv);
-        tmem_ld_wait();
-        if (diag) {
+      for (int c = 0; c < NC; ++c) {
+        float (&s32)[32] = sv[c];
+        if constexpr (PARTS > 1) {
+          tmem_ld32(s_col + c * 32, s32);
+          tmem_ld_wait();
+          if (diag) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if ((half * C::COLS + c * 32 + e) > r) sv[e] = -INFINITY;
+            for (int e = 0; e < 32; ++e)
+              if ((half * C::COLS + c * 32 + e) > r) s32[e] = -INFINITY;
+          }
         }
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           float x0, x1;
-          f2_unpack(f2_fma(f2_pack(sv[2 * e], sv[2 * e + 1]), sl2x2, nmx2), x0, x1);
+          f2_unpack(f2_fma(f2_pack(s32[2 * e], s32[2 * e + 1]), sl2x2, nmx2), x0, x1);
           const float p0 = ex2_approx(x0);
           const float p1 = ex2_approx(x1);
           r4[e & 3] = f2_add(r4[e & 3], f2_pack(p0, p1));

@@ -146,7 +146,7 @@ std::atomic<int> g_attn64[kMaxDevices], g_attn128[kMaxDevices], g_gath64[kMaxDev
     g_select[kMaxDevices];
 
 // Softmax warpgroups per 128-row query tile in the attention kernel.
-constexpr int kSoftmaxParts = 2;
+constexpr int kSoftmaxParts = 1;
 
 constexpr int kBudgetSmem = tsa::BS_WARPS * 256 * (8 + 4);
 constexpr int kSelectSmem = tsa::BS_WARPS * 256 * 4;
