@@ -349,7 +349,7 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
     cflops = compressed_flops(wl, ks)
     attn_ms = stage_ms["attend"]
     achieved = cflops / (attn_ms * 1e-3) / 1e12
-    roof = {"bound": "tensor", "kernel": "attend2_kernel<128,2,false,true> (attention + scatter epilogue)",
+    roof = {"bound": "tensor", "kernel": "attend2_kernel<128,false,true> (attention + scatter epilogue)",
             "achieved": achieved,
             "peak": pk["bf16_sustained"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_sustained"],
             "traffic": ATTN_DRAM_BYTES_PER_KEPT_ROW * wl.Hq * sum(ks),

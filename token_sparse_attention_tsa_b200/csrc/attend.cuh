@@ -41,25 +41,19 @@ struct AttnArgs {
 };
 
 // ---------------------------------------------------------------------------
-// Two query tiles per CTA (rows [256c, 256c+256) of one head), ping-ponged,
-// with PARTS softmax warpgroups per tile (each row's 128 S columns split in
-// PARTS parts):
-//   warps 0..4*PARTS-1          softmax of query tile 0 (warp w: rows
-//                               32(w%4)..+32, part w/4)
-//   warps 4*PARTS..8*PARTS-1    softmax of query tile 1 (same split)
-//   warp 8*PARTS                TMEM allocator + MMA issuer
-//   warp 8*PARTS+1              TMA producer
-// PARTS = 1 is the configuration in use: one thread owns a whole row, holds
-// its 128 S values in registers between the max and the exponentials, and
-// needs no exchange.  With PARTS = 2 (18 warps, so at most 96 registers a
-// thread) each row's max and sum are combined across its two halves through
-// shared memory behind a named barrier of the tile's 256 threads that also
-// ANDs the threads' progress flags, so both halves always take the same
-// branch, and S is re-read from TMEM for the exponentials.
-// TMEM: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D, 256+2D).  Each
-// part writes its P values (bf16, two per 32-bit column) over the first half
-// of its own S columns, and the P.V MMA reads P from TMEM, so P never touches
-// shared memory.  K and V
+// Two query tiles per CTA (rows [256c, 256c+256) of one head), ping-ponged:
+//   warps 0..3   softmax of query tile 0 (warp w: rows 32w..32w+31, one
+//                thread per row, all 128 S columns of its row)
+//   warps 4..7   softmax of query tile 1 (same split)
+//   warp 8       TMEM allocator + MMA issuer
+//   warp 9       TMA producer
+// TMEM: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D, 256+2D).  A
+// softmax thread reads its 128 S values into registers once, takes the row
+// max, and writes its P values (bf16, two per 32-bit column) over the first
+// 64 of its tile's S columns; the P.V MMA reads P from TMEM, so P never
+// touches shared memory.  P is released to the MMA warp in P_SPLITS column
+// groups (one barrier each), so the first k-steps of P.V run while the
+// softmax still computes the later columns.  K and V
 // tiles stream through one TMA ring of NSLOT slots in the order K0 V0 K1 V1 ...
 // Per KV tile j the MMA warp issues S0_j, PV1_{j-1}, S1_j, PV0_j: while one
 // tile's softmax runs the tensor core works on the other tile.  S0_{j+1}
@@ -67,12 +61,11 @@ struct AttnArgs {
 // the same thread; tcgen05.mma ops of one thread execute in issue order, so
 // the read precedes the overwrite (the same reliance as the open CUTLASS
 // sm100 attention mainloop).
-template <int D, int PARTS>
+template <int D>
 struct Attn2Layout {
   static constexpr int BM = 128;
   static constexpr int BN = 128;
-  static constexpr int SOFT_WARPS = 8 * PARTS;        // 4 warps per part per tile
-  static constexpr int COLS = BN / PARTS;              // S columns per softmax thread
+  static constexpr int SOFT_WARPS = 8;
   static constexpr int THREADS = (SOFT_WARPS + 2) * 32;
   static constexpr int MMA_WARP = SOFT_WARPS;
   static constexpr int LOAD_WARP = SOFT_WARPS + 1;
@@ -80,12 +73,12 @@ struct Attn2Layout {
   static constexpr int NCH = D / 64;
   static constexpr int TILE = 128 * D * 2;            // bytes of one Q, K or V tile
   static constexpr int NSLOT = D == 128 ? 4 : 9;      // K/V ring slots
+  static constexpr int P_SPLITS = 2;                  // P released in this many column groups
+  static constexpr int KSTEPS = BN / 16;              // P.V k-steps per KV tile
   static constexpr int OFF_Q0 = 0;
   static constexpr int OFF_Q1 = TILE;
   static constexpr int OFF_RING = 2 * TILE;
-  static constexpr int OFF_X = OFF_RING + NSLOT * TILE;        // row max / sum exchange
-  static constexpr int X_BYTES = 2 * 2 * 2 * 128 * 4;          // [parity][tile][half][row]
-  static constexpr int OFF_BAR = OFF_X + X_BYTES;
+  static constexpr int OFF_BAR = OFF_RING + NSLOT * TILE;
   static constexpr int TOTAL = OFF_BAR + 512;
   static constexpr int ALLOC = (TOTAL + 1024) > 120 * 1024 ? (TOTAL + 1024) : 120 * 1024;
   static constexpr int TMEM_COLS = 512;
@@ -95,10 +88,12 @@ struct Attn2Layout {
   static constexpr int B_FULL = 1;                    // + slot
   static constexpr int B_EMPTY = 1 + NSLOT;           // + slot
   static constexpr int B_S = 1 + 2 * NSLOT;           // + tile (S ready)
-  static constexpr int B_P = B_S + 2;                 // + tile (P written)
-  static constexpr int B_PV = B_P + 2;                // + tile (P.V complete)
+  static constexpr int B_P = B_S + 2;                 // + tile * P_SPLITS + group (P written)
+  static constexpr int B_PV = B_P + 2 * P_SPLITS;     // + tile (P.V complete)
   static constexpr int B_DRAIN = B_PV + 2;
   static constexpr int B_COUNT = B_DRAIN + 1;
+  static_assert(8 * B_COUNT + 8 <= 512, "barrier area");
+  static_assert(KSTEPS % P_SPLITS == 0 && (BN / 32) % P_SPLITS == 0, "P groups");
 };
 
 // kGather: Q, K and V rows are gathered by index (tile::gather4 from 2D maps
@@ -108,11 +103,11 @@ struct Attn2Layout {
 // pass before the kernel is faster when compressed buffers can be held.)
 // kScatter: output row i is written to row idx[i] of o (in place in the
 // full-length output) instead of row i of a compressed output.
-template <int D, int PARTS, bool kGather, bool kScatter>
-__global__ void __launch_bounds__(Attn2Layout<D, PARTS>::THREADS, 1)
+template <int D, bool kGather, bool kScatter>
+__global__ void __launch_bounds__(Attn2Layout<D>::THREADS, 1)
     attend2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
-  using C = Attn2Layout<D, PARTS>;
+  using C = Attn2Layout<D>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -147,7 +142,7 @@ __global__ void __launch_bounds__(Attn2Layout<D, PARTS>::THREADS, 1)
     }
     for (int t = 0; t < 2; ++t) {
       mbar_init(bar(C::B_S + t), 1);
-      mbar_init(bar(C::B_P + t), 4 * PARTS);      // one arrival per softmax warp
+      for (int g = 0; g < C::P_SPLITS; ++g) mbar_init(bar(C::B_P + t * C::P_SPLITS + g), 4);  // one arrival per warp
       mbar_init(bar(C::B_PV + t), 1);
     }
     mbar_init(bar(C::B_DRAIN), 1);
@@ -252,20 +247,6 @@ __global__ void __launch_bounds__(Attn2Layout<D, PARTS>::THREADS, 1)
           mma_commit(bar(C::B_S + t));
         }
       };
-      auto issue_pv = [&](int t, int j) {
-        const uint64_t dv = dv0 + static_cast<uint64_t>((slot_of(2 * j + 1) * C::TILE) >> 4);
-        if (leader) {
-#pragma unroll
-          for (int kk = 0; kk < C::BN / 16; ++kk) {
-            // P of keys [16kk, 16kk+16): part p = 16kk / COLS holds them from
-            // column p*COLS, two keys per column.
-            const uint32_t pcol = (16 * kk / C::COLS) * C::COLS + (16 * kk % C::COLS) / 2;
-            mma_bf16_ts(tmem + C::TMEM_O + t * D, tmem + t * 128 + pcol,
-                        dv + static_cast<uint64_t>((kk * 2048) >> 4), idO, (j > 0 || kk > 0) ? 1u : 0u);
-          }
-          mma_commit(bar(C::B_PV + t));
-        }
-      };
       auto commit_to = [&](uint32_t br) {
         if (leader) mma_commit(br);
       };
@@ -273,21 +254,38 @@ __global__ void __launch_bounds__(Attn2Layout<D, PARTS>::THREADS, 1)
         return __all_sync(0xffffffffu, mbar_wait(br, par, wc));
       };
       auto full = [&](int n) { return wait_all(bar(C::B_FULL + slot_of(n)), use_of(n) & 1); };
+      // O_t += P_t,j V_j, one group of k-steps per released P group.  P of
+      // keys [16kk, 16kk+16) sits in TMEM column 8kk of the tile's S columns.
+      auto issue_pv = [&](int t, int j) -> bool {
+        const uint64_t dv = dv0 + static_cast<uint64_t>((slot_of(2 * j + 1) * C::TILE) >> 4);
+        constexpr int KPG = C::KSTEPS / C::P_SPLITS;
+#pragma unroll
+        for (int g = 0; g < C::P_SPLITS; ++g) {
+          if (!wait_all(bar(C::B_P + t * C::P_SPLITS + g), j & 1)) return false;
+          tc_fence_after();
+          if (leader) {
+#pragma unroll
+            for (int kk = g * KPG; kk < (g + 1) * KPG; ++kk)
+              mma_bf16_ts(tmem + C::TMEM_O + t * D, tmem + t * 128 + 8 * kk,
+                          dv + static_cast<uint64_t>((kk * 2048) >> 4), idO, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+        commit_to(bar(C::B_PV + t));
+        return true;
+      };
+      // The waits for K_{j+1} and V_j come before the P waits of PV0_j: those
+      // tiles have normally landed long before, and once P0_j is released
+      // PV0_j and S0_{j+1} go out back to back.  Every slot these loads need
+      // was released by a commit issued earlier in this loop, so waiting for
+      // them here cannot deadlock the ring.
       // test hook: phase 0 of the drain barrier completes only at teardown,
       // so this bounded wait runs out and takes the abort path
-      // The waits for K_{j+1} and V_j come before the wait for P0_j: those
-      // tiles have normally landed long before, and once P0_j arrives PV0_j
-      // and S0_{j+1} go out back to back.  Every slot these loads need was
-      // released by a commit issued earlier in this loop, so waiting for them
-      // here cannot deadlock the ring.
       bool ok = !(a.test_stall && !wait_all(bar(C::B_DRAIN), 0)) && wait_all(bar(C::B_Q), 0) && full(0);
       for (int j = 0; ok && j < n_kv; ++j) {
         tc_fence_after();                                                // K_j has landed
         if (j <= last0) issue_s(0, j);
         if (two && j >= 1) {
-          if (!(ok = wait_all(bar(C::B_P + 1), (j - 1) & 1))) break;
-          tc_fence_after();
-          issue_pv(1, j - 1);
+          if (!(ok = issue_pv(1, j - 1))) break;
           commit_to(bar(C::B_EMPTY + slot_of(2 * j - 1)));               // V_{j-1} done
         }
         if (two) issue_s(1, j);
@@ -296,9 +294,7 @@ __global__ void __launch_bounds__(Attn2Layout<D, PARTS>::THREADS, 1)
         if (j <= last0) {
           if (!(ok = full(2 * j + 1))) break;                            // V_j
           if (more && !(ok = full(2 * j + 2))) break;                    // K_{j+1}
-          if (!(ok = wait_all(bar(C::B_P + 0), j & 1))) break;
-          tc_fence_after();
-          issue_pv(0, j);
+          if (!(ok = issue_pv(0, j))) break;
           if (!two) commit_to(bar(C::B_EMPTY + slot_of(2 * j + 1)));
         } else if (more && !(ok = full(2 * j + 2))) {
           break;
@@ -306,72 +302,50 @@ __global__ void __launch_bounds__(Attn2Layout<D, PARTS>::THREADS, 1)
       }
       if (ok && two) {
         const int j = n_kv - 1;
-        if (wait_all(bar(C::B_P + 1), j & 1) && full(2 * j + 1)) {
-          tc_fence_after();
-          issue_pv(1, j);
-          commit_to(bar(C::B_EMPTY + slot_of(2 * j + 1)));
-        }
+        if (full(2 * j + 1) && issue_pv(1, j)) commit_to(bar(C::B_EMPTY + slot_of(2 * j + 1)));
       }
       commit_to(bar(C::B_DRAIN));
       if (leader) mbar_wait_drain(bar(C::B_DRAIN), 0, 1000000000ull);
     }
-  } else if (run && (warp < C::SOFT_WARPS / 2 || two)) {
+  } else if (run && warp < C::SOFT_WARPS && (warp < 4 || two)) {
     // ------------------------------------------------------------ softmax
-    const int tt = warp / (4 * PARTS);           // query tile of this warp
-    const int half = (warp >> 2) % PARTS;        // columns [COLS*half, COLS*half+COLS)
+    const int tt = warp >> 2;                    // query tile of this warp
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;                // row within the tile
     const int tile = t0 + tt;
     const int row = tile * C::BM + r;
     const int last = tile;                       // its diagonal KV tile
     const bool last_active = tt == (two ? 1 : 0);
-    const uint32_t named = 1 + tt;               // named barrier of the tile's 256 threads
     const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
-    const uint32_t s_col = tmem + lane_off + tt * 128 + half * C::COLS;
-    const uint32_t p_col = s_col;                // P over the first COLS/2 of the part's columns
-    const uint32_t o_col = tmem + lane_off + C::TMEM_O + tt * D + half * (D / PARTS);
-    float* xch = reinterpret_cast<float*>(gbase + C::OFF_X);   // [parity][tile][half][row]
-    auto xidx = [&](int par, int hf) { return ((par * 2 + tt) * 2 + hf) * 128 + r; };
+    const uint32_t s_col = tmem + lane_off + tt * 128;
+    const uint32_t o_col = tmem + lane_off + C::TMEM_O + tt * D;
     const float sl2 = a.scale_log2;
     float m_used = -INFINITY;
-    float l = 0.f;                               // this half's share of the row sum
+    float l = 0.f;
     bool live = true;
     for (int j = 0; j <= last; ++j) {
-      live = live && __all_sync(0xffffffffu, mbar_wait(bar(C::B_S + tt), j & 1, wc));
-      float mh = -INFINITY;
+      if (!(live = __all_sync(0xffffffffu, mbar_wait(bar(C::B_S + tt), j & 1, wc)))) break;
+      tc_fence_after();
       const bool diag = (j == last);
-      constexpr int NC = C::COLS / 32;
-      float sv[NC][32];
-      if (live) {  // pass 1: this part's row max
-        tc_fence_after();
+      float sv[4][32];
 #pragma unroll
-        for (int c = 0; c < NC; ++c) tmem_ld32(s_col + c * 32, sv[c]);
-        tmem_ld_wait();
-        if (diag) {  // causal mask, only on the diagonal tile
+      for (int c = 0; c < 4; ++c) tmem_ld32(s_col + c * 32, sv[c]);
+      tmem_ld_wait();
+      if (diag) {  // causal mask, only on the diagonal tile
 #pragma unroll
-          for (int c = 0; c < NC; ++c)
+        for (int c = 0; c < 4; ++c)
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if ((half * C::COLS + c * 32 + e) > r) sv[c][e] = -INFINITY;
-        }
-        // row max: four chains of three-input maxima over value pairs
-        float m4[4] = {sv[0][0], sv[0][1], sv[0][2], sv[0][3]};
-#pragma unroll
-        for (int i = 4; i < C::COLS; i += 2) {       // i even: i, i+1 lie in one 32-chunk
-          const int u = (i >> 1) & 3;
-          m4[u] = fmax3(m4[u], sv[i >> 5][i & 31], sv[i >> 5][(i & 31) + 1]);
-        }
-        mh = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
+          for (int e = 0; e < 32; ++e)
+            if (c * 32 + e > r) sv[c][e] = -INFINITY;
       }
-      float mx = mh;
-      if constexpr (PARTS == 2) {
-        xch[xidx(j & 1, half)] = mh;
-        live = bar_and(named, 256, live);        // both halves agree to go on
-        if (!live) continue;                     // keep the barrier count uniform
-        mx = fmaxf(mh, xch[xidx(j & 1, half ^ 1)]);
-      } else {
-        if (!live) continue;
+      // row max: four chains of three-input maxima over value pairs
+      float m4[4] = {sv[0][0], sv[0][1], sv[0][2], sv[0][3]};
+#pragma unroll
+      for (int i = 4; i < C::BN; i += 2) {       // i even: i, i+1 lie in one 32-chunk
+        const int u = (i >> 1) & 3;
+        m4[u] = fmax3(m4[u], sv[i >> 5][i & 31], sv[i >> 5][(i & 31) + 1]);
       }
+      const float mx = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
       const float m_new = fmaxf(m_used, mx * sl2);
       const bool resc = m_new > m_used + 8.0f;   // lazy rescale (factor <= 2^8 tolerated)
       const float alpha = resc ? ex2_approx(m_used - m_new) : 1.f;
@@ -381,51 +355,40 @@ __global__ void __launch_bounds__(Attn2Layout<D, PARTS>::THREADS, 1)
       uint64_t r4[4];                               // packed partial row sums
 #pragma unroll
       for (int u = 0; u < 4; ++u) r4[u] = 0ull;
-      // pass 2: S columns [32c, 32c+32) of the part give P columns
-      // [16c, 16c+16), which lie in columns already read.  A thread that
-      // owns a whole row still holds its S values from pass 1; with the row
-      // split in parts the register budget only allows re-reading them.
+      // S columns [32c, 32c+32) give P columns [16c, 16c+16); every S value
+      // is already in registers, so P may overwrite any S column.
+      constexpr int CPG = 4 / C::P_SPLITS;          // 32-column chunks per P group
 #pragma unroll
-      for (int c = 0; c < NC; ++c) {
-        float (&s32)[32] = sv[c];
-        if constexpr (PARTS > 1) {
-          tmem_ld32(s_col + c * 32, s32);
-          tmem_ld_wait();
-          if (diag) {
+      for (int g = 0; g < C::P_SPLITS; ++g) {
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if ((half * C::COLS + c * 32 + e) > r) s32[e] = -INFINITY;
+        for (int cc = 0; cc < CPG; ++cc) {
+          const int c = g * CPG + cc;
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(sv[c][2 * e], sv[c][2 * e + 1]), sl2x2, nmx2), x0, x1);
+            const float p0 = ex2_approx(x0);
+            const float p1 = ex2_approx(x1);
+            r4[e & 3] = f2_add(r4[e & 3], f2_pack(p0, p1));
+            pk[e] = pack_bf16x2(p0, p1);
           }
+          tmem_st16u(s_col + c * 16, pk);
         }
-        uint32_t pk[16];
+        if (g == 0) {
+          // Before the first P group is released: O is rescaled when a
+          // row's max grew past the lazy threshold, and V rows past `valid`
+          // are zeroed (those rows may carry any bits; their P weights are 0
+          // but 0 * NaN would poison O).  P.V j-1 has completed by now, as
+          // S_j was committed after it, so the PV wait returns at once; the
+          // PV barrier can never be two phases ahead here because P.V j
+          // needs this tile's P first, so a parity wait after skipped ones
+          // still names the right phase.
+          if (j > 0 && __any_sync(0xffffffffu, resc)) {
+            if (!(live = __all_sync(0xffffffffu, mbar_wait(bar(C::B_PV + tt), (j - 1) & 1, wc)))) break;
+            tc_fence_after();
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          float x0, x1;
-          f2_unpack(f2_fma(f2_pack(s32[2 * e], s32[2 * e + 1]), sl2x2, nmx2), x0, x1);
-          const float p0 = ex2_approx(x0);
-          const float p1 = ex2_approx(x1);
-          r4[e & 3] = f2_add(r4[e & 3], f2_pack(p0, p1));
-          pk[e] = pack_bf16x2(p0, p1);
-        }
-        tmem_st16u(p_col + c * 16, pk);
-      }
-      float rs[8];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) f2_unpack(r4[u], rs[2 * u], rs[2 * u + 1]);
-      l = l * alpha + (((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7])));
-      // O is rescaled only when a row's max grew past the lazy threshold, and
-      // then only once the previous P.V into O has completed (and before this
-      // tile's P.V, which waits for P_FULL).  Otherwise the wait is skipped:
-      // P.V MMAs into one accumulator run in issue order.  The PV barrier can
-      // never be two phases ahead here (P.V j needs this tile's P first), so a
-      // parity wait after skipped ones still names the right phase.
-      if (j > 0 && __any_sync(0xffffffffu, resc)) {
-        live = __all_sync(0xffffffffu, mbar_wait(bar(C::B_PV + tt), (j - 1) & 1, wc));
-        if (live) {
-          tc_fence_after();
-          {
-#pragma unroll
-            for (int c = 0; c < D / PARTS / 32; ++c) {
+            for (int c = 0; c < D / 32; ++c) {
               float ov[32];
               tmem_ld32(o_col + c * 32, ov);
               tmem_ld_wait();
@@ -434,43 +397,38 @@ __global__ void __launch_bounds__(Attn2Layout<D, PARTS>::THREADS, 1)
               tmem_st32(o_col + c * 32, ov);
             }
           }
-        }
-      }
-      // Rows of the KV tile that holds `valid` may carry any bits beyond it;
-      // their P weights are 0 but 0 * NaN would poison O, so zero them.
-      if (live && half == 0 && diag && last_active && (j * C::BN + C::BN > valid)) {
-        const int n = 2 * j + 1;
-        live = __all_sync(0xffffffffu, mbar_wait(bar(C::B_FULL + slot_of(n)), use_of(n) & 1, wc));
-        if (live && j * C::BN + r >= valid) {
+          if (diag && last_active && (j * C::BN + C::BN > valid)) {
+            const int n = 2 * j + 1;
+            if (!(live = __all_sync(0xffffffffu, mbar_wait(bar(C::B_FULL + slot_of(n)), use_of(n) & 1, wc)))) break;
+            if (j * C::BN + r >= valid) {
 #pragma unroll
-          for (int c = 0; c < C::NCH; ++c) {
-            uint4* vrow = reinterpret_cast<uint4*>(gbase + C::OFF_RING + slot_of(n) * C::TILE + c * C::CHUNK + r * 128);
+              for (int c = 0; c < C::NCH; ++c) {
+                uint4* vrow = reinterpret_cast<uint4*>(gbase + C::OFF_RING + slot_of(n) * C::TILE + c * C::CHUNK + r * 128);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) vrow[e] = make_uint4(0, 0, 0, 0);
+                for (int e = 0; e < 8; ++e) vrow[e] = make_uint4(0, 0, 0, 0);
+              }
+            }
+            fence_proxy_async_smem();
           }
         }
-        fence_proxy_async_smem();
-      }
-      if (live) {
-        // the warp's TMEM stores (and V zeroing) are complete; one lane
-        // arrives for the warp
+        // the warp's TMEM stores (O rescale, P) and V zeroing are complete;
+        // one lane arrives for the warp
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(bar(C::B_P + tt));
+        if (lane == 0) mbar_arrive(bar(C::B_P + tt * C::P_SPLITS + g));
       }
+      if (!live) break;                            // a wait above ran out
+      float rs[8];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) f2_unpack(r4[u], rs[2 * u], rs[2 * u + 1]);
+      l = l * alpha + (((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7])));
     }
     // ------------------------------------------------------------ epilogue
     live = live && __all_sync(0xffffffffu, mbar_wait(bar(C::B_PV + tt), last & 1, wc));
-    float lt = l;
-    if constexpr (PARTS == 2) {
-      xch[xidx(0, half)] = l;  // parity-0 slots are free: every read of them is behind us
-      live = bar_and(named, 256, live);
-      if (live) lt = l + xch[xidx(0, half ^ 1)];
-    }
     if (live) {
       tc_fence_after();
-      const float inv_l = 1.f / lt;
+      const float inv_l = 1.f / l;
       int orow_index = row;
       bool store = row < valid;
       if constexpr (kScatter) {  // compressed row i goes to token S_h[i]
@@ -480,9 +438,9 @@ __global__ void __launch_bounds__(Attn2Layout<D, PARTS>::THREADS, 1)
           if (a.status) atomicOr(a.status, 0x4u);
         }
       }
-      __nv_bfloat16* orow = a.o + (static_cast<size_t>(bh) * a.L + (store ? orow_index : 0)) * D + half * (D / PARTS);
+      __nv_bfloat16* orow = a.o + (static_cast<size_t>(bh) * a.L + (store ? orow_index : 0)) * D;
 #pragma unroll
-      for (int c = 0; c < D / PARTS / 32; ++c) {
+      for (int c = 0; c < D / 32; ++c) {
         float ov[32];
         tmem_ld32(o_col + c * 32, ov);
         tmem_ld_wait();
@@ -499,8 +457,8 @@ __global__ void __launch_bounds__(Attn2Layout<D, PARTS>::THREADS, 1)
           }
         }
       }
-      if (a.lse && half == 0 && row < valid)
-        a.lse[static_cast<size_t>(bh) * a.L + row] = (m_used + __log2f(lt)) * 0.69314718055994531f;
+      if (a.lse && row < valid)
+        a.lse[static_cast<size_t>(bh) * a.L + row] = (m_used + __log2f(l)) * 0.69314718055994531f;
     }
   }
 

@@ -145,9 +145,6 @@ std::atomic<int> g_attn64[kMaxDevices], g_attn128[kMaxDevices], g_gath64[kMaxDev
     g_st128[kMaxDevices], g_sum64[kMaxDevices], g_sum128[kMaxDevices], g_budget[kMaxDevices],
     g_select[kMaxDevices];
 
-// Softmax warpgroups per 128-row query tile in the attention kernel.
-constexpr int kSoftmaxParts = 1;
-
 constexpr int kBudgetSmem = tsa::BS_WARPS * 256 * (8 + 4);
 constexpr int kSelectSmem = tsa::BS_WARPS * 256 * 4;
 
@@ -305,17 +302,16 @@ tsa_status run_attend(const tsa_params* p, const void* q, const void* k, const v
     kernel<<<grid, threads, smem, st>>>(mq, mk, mv, a);
     return launch_ok();
   };
-  constexpr int P = kSoftmaxParts;
   if (p->d == 128) {
-    using L = tsa::Attn2Layout<128, P>;
-    if (!scatter) return launch(tsa::attend2_kernel<128, P, false, false>, g_attn128, L::THREADS, L::ALLOC);
-    if (!gather) return launch(tsa::attend2_kernel<128, P, false, true>, g_gq128, L::THREADS, L::ALLOC);
-    return launch(tsa::attend2_kernel<128, P, true, true>, g_gath128, L::THREADS, L::ALLOC);
+    using L = tsa::Attn2Layout<128>;
+    if (!scatter) return launch(tsa::attend2_kernel<128, false, false>, g_attn128, L::THREADS, L::ALLOC);
+    if (!gather) return launch(tsa::attend2_kernel<128, false, true>, g_gq128, L::THREADS, L::ALLOC);
+    return launch(tsa::attend2_kernel<128, true, true>, g_gath128, L::THREADS, L::ALLOC);
   }
-  using L = tsa::Attn2Layout<64, P>;
-  if (!scatter) return launch(tsa::attend2_kernel<64, P, false, false>, g_attn64, L::THREADS, L::ALLOC);
-  if (!gather) return launch(tsa::attend2_kernel<64, P, false, true>, g_gq64, L::THREADS, L::ALLOC);
-  return launch(tsa::attend2_kernel<64, P, true, true>, g_gath64, L::THREADS, L::ALLOC);
+  using L = tsa::Attn2Layout<64>;
+  if (!scatter) return launch(tsa::attend2_kernel<64, false, false>, g_attn64, L::THREADS, L::ALLOC);
+  if (!gather) return launch(tsa::attend2_kernel<64, false, true>, g_gq64, L::THREADS, L::ALLOC);
+  return launch(tsa::attend2_kernel<64, true, true>, g_gath64, L::THREADS, L::ALLOC);
 }
 
 // Zero the rows of o that no index selects (the selected rows are left as
