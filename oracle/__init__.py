@@ -28,9 +28,15 @@ Readings taken where the page is silent (each is also pinned by a test):
     Tokens are taken in ascending q order; the pruned count p_h is the
     largest p whose first-p prefix sum stays <= T (the token that would
     push the pruned mass past tau is kept).  k_h = L - p_h.
-  * the "global budget" is per sequence: k_b = max over heads of k_h.
-  * per-head top-k: the k_b indices with the largest fp32 score, equal
-    scores broken toward the smaller index, emitted in ascending order.
+  * the "global budget" is per sequence: k_b = max over heads of k_h
+    (budget mode "max", the default).  Two variants the page leaves open:
+    "mean" keeps k_b = ceil(mean over heads of k_h) in every head, and
+    "per_head" keeps k_h in head h (no budget shared across heads).
+  * optional forced keeps: with keep_recent = r, the last r tokens of the
+    sequence are kept in every head; each k_h is raised to at least r, and
+    the forced tokens rank above every score in the selection.
+  * per-head top-k: the kept-count indices with the largest fp32 score,
+    equal scores broken toward the smaller index, emitted in ascending order.
   * compressed causality: compressed row i attends compressed keys j <= i;
     since indices ascend, this is the original causal order.
   * GQA: selection per Q head h; K and V rows come from KV head h // G.
@@ -130,15 +136,40 @@ def pruned_count_head(scores_head: np.ndarray, tau: float) -> int:
     return int(np.count_nonzero(cum <= T))  # cum is non-decreasing
 
 
-def coverage_budget(scores: np.ndarray, tau: float):
-    """Per-head keep counts k_h = L - p_h [B,Hq] and per-sequence k_b [B]."""
+BUDGET_MODES = ("max", "mean", "per_head")
+
+
+def coverage_budget(scores: np.ndarray, tau: float, mode: str = "max", keep_recent: int = 0):
+    """Per-head keep counts k_h = max(L - p_h, r) [B,Hq] and the sequence
+    budget k_b [B]: max over the heads ("max" and "per_head") or the ceiling
+    of their mean ("mean").  r = keep_recent clipped to [0, L]."""
+    if mode not in BUDGET_MODES:
+        raise ValueError(mode)
     B, Hq, L = scores.shape
+    r = min(max(int(keep_recent), 0), L)
     k_head = np.empty((B, Hq), dtype=np.int32)
     for b in range(B):
         for h in range(Hq):
-            k_head[b, h] = L - pruned_count_head(scores[b, h], tau)
-    k_seq = k_head.max(axis=1).astype(np.int32)   # global budget of the sequence
-    return k_head, k_seq
+            k_head[b, h] = max(L - pruned_count_head(scores[b, h], tau), r)
+    if mode == "mean":
+        k_seq = -(-k_head.astype(np.int64).sum(axis=1) // Hq)   # ceiling of the mean
+    else:
+        k_seq = k_head.max(axis=1)                           # global budget of the sequence
+    return k_head, k_seq.astype(np.int32)
+
+
+def kept_counts(k_head: np.ndarray, k_seq: np.ndarray, mode: str = "max") -> np.ndarray:
+    """Rows kept by every head [B,Hq]: its own k_h in "per_head" mode, else
+    the sequence budget k_b."""
+    if mode == "per_head":
+        return np.asarray(k_head, dtype=np.int32).copy()
+    return np.repeat(np.asarray(k_seq, dtype=np.int32)[:, None], k_head.shape[1], axis=1)
+
+
+def _kept(kept: np.ndarray, b: int, h: int) -> int:
+    """Kept rows of head (b, h) from per-sequence [B] or per-head [B,Hq] counts."""
+    kept = np.asarray(kept)
+    return int(kept[b] if kept.ndim == 1 else kept[b, h])
 
 
 # ---------------------------------------------------------------------------
@@ -146,21 +177,26 @@ def coverage_budget(scores: np.ndarray, tau: float):
 # [GS] "Cobertura Dinamica de Tokens", per-head selection bullet, and
 # "Arquitectura Central", compression step.
 # ---------------------------------------------------------------------------
-def select_head(scores_head: np.ndarray, k: int) -> np.ndarray:
+def select_head(scores_head: np.ndarray, k: int, keep_recent: int = 0) -> np.ndarray:
+    """The k best tokens, ascending: the last keep_recent tokens first, then
+    score descending, then index ascending."""
     L = scores_head.shape[0]
     s = np.asarray(scores_head, dtype=np.float32).astype(np.float64)
-    order = np.lexsort((np.arange(L), -s))     # score descending, index ascending
+    not_forced = np.arange(L) < L - min(max(int(keep_recent), 0), L)
+    order = np.lexsort((np.arange(L), -s, not_forced))
     return np.sort(order[:k]).astype(np.int32)
 
 
-def select_topk(scores: np.ndarray, k_seq: np.ndarray) -> np.ndarray:
-    """idx [B,Hq,L] int32: first k_b entries are S_h ascending, the rest -1."""
+def select_topk(scores: np.ndarray, kept: np.ndarray, keep_recent: int = 0) -> np.ndarray:
+    """idx [B,Hq,L] int32: the first k entries of head (b, h) are S_h
+    ascending, the rest -1; k comes from kept ([B] per sequence or [B,Hq]
+    per head)."""
     B, Hq, L = scores.shape
     idx = np.full((B, Hq, L), -1, dtype=np.int32)
     for b in range(B):
         for h in range(Hq):
-            kb = int(k_seq[b])
-            idx[b, h, :kb] = select_head(scores[b, h], kb)
+            kb = _kept(kept, b, h)
+            idx[b, h, :kb] = select_head(scores[b, h], kb, keep_recent)
     return idx
 
 
@@ -168,15 +204,16 @@ def select_topk(scores: np.ndarray, k_seq: np.ndarray) -> np.ndarray:
 # Step 4: gather into dense compressed tensors.  [GS] "Arquitectura Central".
 # ---------------------------------------------------------------------------
 def gather_qkv(q, k, v, idx, k_seq):
-    """Compressed copies (same dtype as the inputs), rows >= k_b left zero."""
+    """Compressed copies (same dtype as the inputs), rows >= k_b left zero.
+    k_seq: kept rows per sequence [B] or per head [B,Hq]."""
     B, Hq, L, d = q.shape
     G = Hq // k.shape[1]
     qc = np.zeros_like(q)
     kc = np.zeros((B, Hq, L, d), dtype=k.dtype)
     vc = np.zeros((B, Hq, L, d), dtype=v.dtype)
     for b in range(B):
-        kb = int(k_seq[b])
         for h in range(Hq):
+            kb = _kept(k_seq, b, h)
             s = idx[b, h, :kb]
             qc[b, h, :kb] = q[b, h, s]
             kc[b, h, :kb] = k[b, h // G, s]
@@ -218,8 +255,8 @@ def compressed_attention(qc, kc, vc, k_seq, scale: float | None = None) -> np.nd
         scale = default_scale(d)
     oc = np.zeros((B, Hq, L, d), dtype=np.float64)
     for b in range(B):
-        kb = int(k_seq[b])
         for h in range(Hq):
+            kb = _kept(k_seq, b, h)
             oc[b, h, :kb] = attention_rows(qc[b, h, :kb], kc[b, h, :kb], vc[b, h, :kb],
                                            np.arange(kb), scale)
     return oc
@@ -247,8 +284,8 @@ def scatter(oc: np.ndarray, idx: np.ndarray, k_seq: np.ndarray, L: int) -> np.nd
     B, Hq, _, d = oc.shape
     o = np.zeros((B, Hq, L, d), dtype=oc.dtype)
     for b in range(B):
-        kb = int(k_seq[b])
         for h in range(Hq):
+            kb = _kept(k_seq, b, h)
             o[b, h, idx[b, h, :kb]] = oc[b, h, :kb]
     return o
 
@@ -256,18 +293,20 @@ def scatter(oc: np.ndarray, idx: np.ndarray, k_seq: np.ndarray, L: int) -> np.nd
 # ---------------------------------------------------------------------------
 # The whole path, step by step.
 # ---------------------------------------------------------------------------
-def forward(q, k, v, w: int, tau: float, scale: float | None = None) -> dict:
+def forward(q, k, v, w: int, tau: float, scale: float | None = None, mode: str = "max",
+            keep_recent: int = 0) -> dict:
     """Scores -> budget -> selection -> gather -> attention -> scatter."""
     B, Hq, L, d = q.shape
     if scale is None:
         scale = default_scale(d)
     scores = proxy_scores(q, k, w, scale)
-    k_head, k_seq = coverage_budget(scores, tau)
-    idx = select_topk(scores, k_seq)
-    qc, kc, vc = gather_qkv(q, k, v, idx, k_seq)
-    oc = compressed_attention(qc, kc, vc, k_seq, scale)
-    o = scatter(oc, idx, k_seq, L)
-    return dict(scores=scores, k_head=k_head, k_seq=k_seq, idx=idx, oc=oc, o=o)
+    k_head, k_seq = coverage_budget(scores, tau, mode, keep_recent)
+    kept = kept_counts(k_head, k_seq, mode)
+    idx = select_topk(scores, kept, keep_recent)
+    qc, kc, vc = gather_qkv(q, k, v, idx, kept)
+    oc = compressed_attention(qc, kc, vc, kept, scale)
+    o = scatter(oc, idx, kept, L)
+    return dict(scores=scores, k_head=k_head, k_seq=k_seq, kept=kept, idx=idx, oc=oc, o=o)
 
 
 def output_rows(q, k, v, idx, k_seq, b: int, h: int, orig_rows, scale: float | None = None):
@@ -278,7 +317,7 @@ def output_rows(q, k, v, idx, k_seq, b: int, h: int, orig_rows, scale: float | N
     G = Hq // k.shape[1]
     if scale is None:
         scale = default_scale(d)
-    kb = int(k_seq[b])
+    kb = _kept(k_seq, b, h)
     s = np.asarray(idx[b, h, :kb], dtype=np.int64)
     orig_rows = np.asarray(orig_rows, dtype=np.int64)
     pos = np.searchsorted(s, orig_rows)
