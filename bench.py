@@ -48,8 +48,12 @@ def dense_flops(wl) -> float:
     return float(wl.B) * wl.Hq * 2.0 * wl.d * wl.L * (wl.L + 1)
 
 
-def compressed_flops(wl, k_seq) -> float:
-    return float(sum(wl.Hq * 2.0 * wl.d * int(k) * (int(k) + 1) for k in k_seq))
+def compressed_flops(wl, kept) -> float:
+    """FLOPs of causal attention over the kept rows: kept is one count per
+    sequence (every head keeps it) or one per (sequence, head)."""
+    kept = np.asarray(kept, dtype=np.float64)
+    per = 2.0 * wl.d * kept * (kept + 1)
+    return float(per.sum() * (wl.Hq if kept.ndim == 1 else 1))
 
 
 def peaks() -> dict:
@@ -144,7 +148,7 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- oracle leg
-def oracle_sample(wl, tau: float, rows: int = 384) -> dict:
+def oracle_sample(wl, tau: float, rows: int = 384, keep_recent: int = 0) -> dict:
     """Time the CPU oracle on a bounded sample of the workload and scale it to
     the whole step: steps 1-4 and 6 for one head at full length, step 5 for
     the `rows` most expensive compressed rows of that head."""
@@ -159,8 +163,8 @@ def oracle_sample(wl, tau: float, rows: int = 384) -> dict:
     scale = O.default_scale(d)
     t0 = time.perf_counter()
     s32 = O.proxy_scores_head(q[0, 0, L - wl.w:], k[0, 0], L, scale)
-    kh = L - O.pruned_count_head(s32, tau)
-    sel = O.select_head(s32, kh)
+    kh = max(L - O.pruned_count_head(s32, tau), keep_recent)
+    sel = O.select_head(s32, kh, keep_recent)
     qc, kc, vc = q[0, 0][sel], k[0, 0][sel], v[0, 0][sel]
     t1 = time.perf_counter()
     r = np.arange(kh - rows, kh)
@@ -183,8 +187,8 @@ def run_reference(args, wl, rank: int) -> int:
     if rank != 0:
         return 0
     for _ in range(args.warmup):
-        oracle_sample(wl, args.tau)
-    runs = [oracle_sample(wl, args.tau) for _ in range(args.steps)]
+        oracle_sample(wl, args.tau, keep_recent=args.keep_recent)
+    runs = [oracle_sample(wl, args.tau, keep_recent=args.keep_recent) for _ in range(args.steps)]
     t = statistics.median(r["seconds_full_step_est"] for r in runs)
     value = dense_flops(wl) / t / 1e12
     line = {
@@ -192,7 +196,7 @@ def run_reference(args, wl, rank: int) -> int:
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "L": wl.L, "d": wl.d,
-                   "w": wl.w, "tau": args.tau},
+                   "w": wl.w, "tau": args.tau, "budget_mode": args.budget_mode, "keep_recent": args.keep_recent},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": runs[0]["cores"], "kind": "oracle",
                          "sample": runs[0]["sample"]},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -230,18 +234,22 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
     pin = [torch.from_numpy(x).view(torch.bfloat16).pin_memory() for x in (qh, kh, vh)]
     q, k, v = [x.to(dev, non_blocking=True) for x in pin]
     o = torch.empty_like(q)
-    p = T.params(wl.B, wl.Hq, wl.Hkv, wl.L, wl.d, wl.w, args.tau)
+    p = T.params(wl.B, wl.Hq, wl.Hkv, wl.L, wl.d, wl.w, args.tau, budget_mode=args.budget_mode,
+                 keep_recent=args.keep_recent)
     ws = T.new_workspace(p, full=True, device=dev)
     scores = torch.empty((wl.B, wl.Hq, wl.L), dtype=torch.float32, device=dev)
     idx = torch.empty((wl.B, wl.Hq, wl.L), dtype=torch.int32, device=dev)
     k_seq = torch.empty((wl.B,), dtype=torch.int32, device=dev)
     k_head = torch.empty((wl.B, wl.Hq), dtype=torch.int32, device=dev)
+    # rows kept per head as the later calls read them: the sequence budget,
+    # or in the per-head mode each head's own count
+    kept = k_head if args.budget_mode == "per_head" else k_seq
     shape = (wl.B, wl.Hq, wl.L, wl.d)
     qc, kc, vc, oc = (torch.empty(shape, dtype=torch.bfloat16, device=dev) for _ in range(4))
     torch.cuda.synchronize()
 
     def forward():
-        T.tsa_forward(p, q, k, v, o, ws, scores, idx, k_seq)
+        T.tsa_forward(p, q, k, v, o, ws, scores, idx, kept)
 
     # the kernels tsa_forward runs, one ABI call each
     stage_names = ["score", "budget", "select", "gather", "attend"]
@@ -252,11 +260,11 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
         evs[1].record(stream)
         T.tsa_budget(p, scores, k_head, k_seq, ws)
         evs[2].record(stream)
-        T.tsa_select(p, scores, k_seq, idx, ws)
+        T.tsa_select(p, scores, kept, idx, ws)
         evs[3].record(stream)
-        T.tsa_gather_qkv(p, q, k, v, idx, k_seq, qc, kc, vc, ws)
+        T.tsa_gather_qkv(p, q, k, v, idx, kept, qc, kc, vc, ws)
         evs[4].record(stream)
-        T.tsa_attend_scatter(p, qc, kc, vc, idx, k_seq, o, None, ws)
+        T.tsa_attend_scatter(p, qc, kc, vc, idx, kept, o, None, ws)
         evs[5].record(stream)
 
     # the separate stage calls the fused attention replaces (attention into a
@@ -266,11 +274,11 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
 
     def unfused(evs):
         evs[0].record(stream)
-        T.tsa_attend(p, qc, kc, vc, k_seq, oc, None, ws)
+        T.tsa_attend(p, qc, kc, vc, kept, oc, None, ws)
         evs[1].record(stream)
-        T.tsa_scatter(p, oc, idx, k_seq, o, ws)
+        T.tsa_scatter(p, oc, idx, kept, o, ws)
         evs[2].record(stream)
-        T.tsa_attend_gathered(p, q, k, v, idx, k_seq, o, None, ws)
+        T.tsa_attend_gathered(p, q, k, v, idx, kept, o, None, ws)
         evs[3].record(stream)
 
     def timed(fn, n):
@@ -293,7 +301,9 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
     with ClockSampler(local_rank) as clk:
         ms = timed(forward, args.steps)
     clocks = clk.summary()
-    ks = k_seq.cpu().numpy().tolist()
+    kept_np = kept.cpu().numpy()
+    ks = kept_np.max(axis=1).tolist() if kept_np.ndim == 2 else kept_np.tolist()
+    kept_rows = int(kept_np.sum()) * (wl.Hq if kept_np.ndim == 1 else 1)
 
     # ---- per-stage breakdown (same kernels, one ABI call per stage)
     def breakdown(fn, names):
@@ -331,7 +341,7 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
         q.copy_(pin[0], non_blocking=True)
         k.copy_(pin[1], non_blocking=True)
         v.copy_(pin[2], non_blocking=True)
-        T.tsa_forward(p, q, k, v, o, ws, scores, idx, k_seq)
+        T.tsa_forward(p, q, k, v, o, ws, scores, idx, kept)
         o_host.copy_(o, non_blocking=True)
 
     e2e_step()
@@ -346,18 +356,18 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
 
     # ---- roofline of the dominant kernel (attention: a dense contraction)
     pk = peaks()
-    cflops = compressed_flops(wl, ks)
+    cflops = compressed_flops(wl, kept_np)
     attn_ms = stage_ms["attend"]
     achieved = cflops / (attn_ms * 1e-3) / 1e12
     roof = {"bound": "tensor", "kernel": "attend2_kernel<128,false,true> (attention + scatter epilogue)",
             "achieved": achieved,
             "peak": pk["bf16_sustained"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_sustained"],
-            "traffic": ATTN_DRAM_BYTES_PER_KEPT_ROW * wl.Hq * sum(ks),
+            "traffic": ATTN_DRAM_BYTES_PER_KEPT_ROW * kept_rows,
             "traffic_note": "ncu DRAM bytes of one launch on the 32K workload, scaled by kept rows",
             "peak_note": f"bf16_tflops_sustained of {pk['source']} peaks (kernel timed inside a long step)"}
     hbm = pk["hbm_gbs"]
     tok = wl.B * wl.Hq * wl.L
-    kept = sum(ks) * wl.Hq
+    kept = kept_rows
     stage_bytes = {
         "gather": kept * wl.d * 2 * 3 * 2,                      # 3 rows read + 3 written
         "scatter": tok * wl.d * 2 + kept * wl.d * 2,            # full write + kept rows read
@@ -370,7 +380,7 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
     value = job_value(wl, world, ms)
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
-        s = oracle_sample(wl, args.tau)
+        s = oracle_sample(wl, args.tau, keep_recent=args.keep_recent)
         cpu = {"value": dense_flops(wl) / s["seconds_full_step_est"] / 1e12, "unit": UNIT, "cores": s["cores"],
                "kind": "oracle", "sample": s["sample"], "sample_seconds": s["sample_seconds"]}
     line = {
@@ -378,9 +388,11 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "L": wl.L, "d": wl.d, "w": wl.w,
-                   "tau": args.tau, "parallelism": f"replicas{world}" if world > 1 else "single",
+                   "tau": args.tau, "budget_mode": args.budget_mode, "keep_recent": args.keep_recent,
+                   "parallelism": f"replicas{world}" if world > 1 else "single",
                    "l2": "inputs larger than L2 (Q 1 GiB, K/V 256 MiB each)"},
         "k_seq": ks, "keep_fraction": [x / wl.L for x in ks],
+        "kept_fraction_all_heads": kept_rows / float(wl.B * wl.Hq * wl.L),
         "dense_ms": dense_ms, "speedup_vs_dense": dense_ms / ms, "sdpa_dense_ms": sdpa_ms,
         "effective_tflops": dense_flops(wl) / (ms * 1e-3) / 1e12,
         "achieved_tflops": cflops / (ms * 1e-3) / 1e12,
@@ -408,6 +420,8 @@ def main() -> int:
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.WORKLOADS))
     ap.add_argument("--impl", default="tsa", choices=["tsa", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--budget-mode", default="max", choices=["max", "mean", "per_head"])
+    ap.add_argument("--keep-recent", type=int, default=0)
     args = ap.parse_args()
     wl = W.WORKLOADS[args.workload]
     if args.tau is None:

@@ -23,6 +23,11 @@
  *   o        bf16 [B, Hq,  L, d]      scores fp32 [B, Hq, L]
  *   idx      int32 [B, Hq, L]: entries [0, k_b) hold S_h ascending, the rest -1
  *   k_head   int32 [B, Hq]            k_seq  int32 [B]
+ *   kept     the rows kept by every head, argument of the calls after the
+ *            budget (named k_seq there): k_seq [B] (one budget per sequence,
+ *            budget modes MAX and MEAN), or the heads' own counts k_head
+ *            [B, Hq] when p->budget_mode == TSA_BUDGET_PER_HEAD.  Below, k_b
+ *            is the kept count of the head in question.
  *   qc, kc, vc, oc  bf16 [B, Hq, L, d]: compressed tensors, capacity L rows
  *            per head, rows [0, k_b) valid (K and V are gathered per query
  *            head, so a GQA group's heads each get their own compressed copy).
@@ -59,7 +64,7 @@
 extern "C" {
 #endif
 
-#define TSA_ABI_VERSION 1
+#define TSA_ABI_VERSION 2
 
 typedef enum tsa_status {
   TSA_OK = 0,
@@ -79,6 +84,15 @@ typedef enum tsa_status {
  * memory and returns without writing outputs.  The context stays usable. */
 #define TSA_FLAG_TEST_STALL 0x80000000u
 
+/* tsa_params.budget_mode: how the heads' coverage counts k_head combine into
+ * the rows each head keeps.  [GS] calls the budget global without saying how
+ * heads combine; MAX (every head of sequence b keeps k_b = max_h k_head) is
+ * the default reading, MEAN (k_b = ceil(mean_h k_head)) and PER_HEAD (head h
+ * keeps its own k_head, no shared budget) are the two other plain ones. */
+#define TSA_BUDGET_MAX 0
+#define TSA_BUDGET_MEAN 1
+#define TSA_BUDGET_PER_HEAD 2
+
 /* Bits of the device status word (first 4 bytes of ws). */
 #define TSA_DEVFLAG_NONFINITE 0x1u
 #define TSA_DEVFLAG_TIMEOUT 0x2u
@@ -91,6 +105,10 @@ typedef struct tsa_params {
   float softmax_scale;  /* 0 selects 1/sqrt(d) (fp32)                        */
   uint32_t flags;       /* 0, or TSA_FLAG_TEST_STALL (failure-path test)     */
   uint32_t timeout_ms;  /* limit of one pipeline wait; 0 selects 2000 ms     */
+  int32_t budget_mode;  /* TSA_BUDGET_MAX (0), _MEAN or _PER_HEAD            */
+  int32_t keep_recent;  /* 0 <= r <= L: the last r tokens of every sequence
+                           are kept in every head (each k_head is raised to
+                           at least r; the selection ranks them first)       */
 } tsa_params;
 
 /* Version of this ABI (TSA_ABI_VERSION of the built library). */
@@ -131,16 +149,19 @@ tsa_status tsa_score(const tsa_params* p, const void* q, const void* k, float* s
  * allocation and per-head selection: per head, masses
  * q_j = ceil(score_j * 2^40) (int64), T = floor(tau * sum_j q_j) (fp64),
  * p_h = the largest count of least-important tokens whose mass sum is <= T,
- * k_head = L - p_h; the sequence's global budget k_seq[b] = max_h k_head.
+ * k_head = max(L - p_h, keep_recent); the sequence's budget k_seq[b] =
+ * max_h k_head (MAX and PER_HEAD modes) or ceil(mean_h k_head) (MEAN).
  * Bit-exact integer arithmetic.  Non-finite scores set TSA_DEVFLAG_NONFINITE.
- * In: scores.  Out: k_head (may be NULL), k_seq.  ws: stage size. */
+ * In: scores.  Out: k_head (may be NULL except in PER_HEAD mode, where it is
+ * the kept-count argument of the later calls), k_seq.  ws: stage size. */
 tsa_status tsa_budget(const tsa_params* p, const float* scores, int32_t* k_head, int32_t* k_seq,
                       void* ws, size_t ws_bytes, void* stream);
 
 /* Step 3 -- per-head top-k.  [GS] "Cobertura Dinamica de Tokens", per-head
- * selection: S_h = the k_seq[b] tokens of largest score, equal scores going
- * to the smaller index, written ascending to idx[b,h,0..k_b); the rest of
- * idx[b,h,:] is set to -1.  In: scores, k_seq.  Out: idx.  ws: stage size. */
+ * selection: S_h = the k_b tokens of largest score (the last keep_recent
+ * tokens first), equal scores going to the smaller index, written ascending
+ * to idx[b,h,0..k_b); the rest of idx[b,h,:] is set to -1.  In: scores,
+ * kept counts (see "kept" above).  Out: idx.  ws: stage size. */
 tsa_status tsa_select(const tsa_params* p, const float* scores, const int32_t* k_seq, int32_t* idx,
                       void* ws, size_t ws_bytes, void* stream);
 
@@ -157,7 +178,7 @@ tsa_status tsa_gather_qkv(const tsa_params* p, const void* q, const void* k, con
 /* Step 5 -- causal attention on the compressed tensors.  [GS] "Arquitectura
  * Central": the compressed tensors stay dense, so an ordinary dense causal
  * kernel runs on them.  oc[b,h,i] = sum_{j<=i} softmax_j(scale *
- * qc[b,h,i].kc[b,h,j]) vc[b,h,j] for i < k_seq[b] (bf16 out, fp32
+ * qc[b,h,i].kc[b,h,j]) vc[b,h,j] for i < k_b (bf16 out, fp32
  * accumulation; tcgen05 tensor cores).  Rows >= k_b of oc are not written.
  * Rows of qc/kc/vc at or beyond k_b may hold any bits.  lse may be NULL.
  * ws: stage size (its status word receives timeouts). */
@@ -205,8 +226,10 @@ tsa_status tsa_scatter(const tsa_params* p, const void* oc, const int32_t* idx, 
 
 /* The whole path: score -> budget -> select -> gather -> attention writing
  * each output row in place, then zeros for the unselected rows (as
- * tsa_attend_scatter); enqueued on stream with no host synchronisation.  scores_out, idx_out, k_seq_out may be NULL (then the
- * workspace holds them); when given they receive the intermediate results.
+ * tsa_attend_scatter); enqueued on stream with no host synchronisation.
+ * scores_out, idx_out, k_seq_out may be NULL (then the workspace holds
+ * them); when given they receive the intermediate results, k_seq_out the
+ * kept counts in the mode's shape ([B], or [B, Hq] in PER_HEAD mode).
  * ws: >= tsa_workspace_size bytes. */
 tsa_status tsa_forward(const tsa_params* p, const void* q, const void* k, const void* v, void* o,
                        float* scores_out, int32_t* idx_out, int32_t* k_seq_out,

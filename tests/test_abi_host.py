@@ -42,7 +42,7 @@ def test_exports_every_declared_symbol(lib):
     assert len(names) == len(T.EXPORTED) and set(names) == set(T.EXPORTED)
     for n in names:
         assert hasattr(lib, n), n
-    assert lib.tsa_abi_version() == 1
+    assert lib.tsa_abi_version() == 2
 
 
 def test_status_strings(lib):
@@ -60,6 +60,9 @@ def test_status_strings(lib):
     (dict(d=96), UNSUPPORTED), (dict(d=256), UNSUPPORTED), (dict(w=4097, L=8192), UNSUPPORTED),
     (dict(L=(1 << 22) + 1, w=1), UNSUPPORTED), (dict(B=64, Hq=64, Hkv=64, L=1 << 20), UNSUPPORTED),
     (dict(d=64), 0), (dict(w=1, L=1), 0), (dict(tau=0.0), 0),
+    (dict(budget_mode=-1), INVALID), (dict(budget_mode=3), INVALID), (dict(budget_mode="mean"), 0),
+    (dict(budget_mode="per_head"), 0), (dict(keep_recent=-1), INVALID), (dict(keep_recent=4097), INVALID),
+    (dict(keep_recent=4096), 0), (dict(keep_recent=64, budget_mode="per_head"), 0),
 ])
 def test_param_validation(lib, kw, want):
     p = good(**kw)
@@ -112,6 +115,15 @@ def test_null_and_misaligned_pointers_rejected(lib):
     assert _call(lib, "tsa_forward", p, FAKE, FAKE, FAKE, FAKE, odd, None, None, FAKE, big, None) == INVALID
     assert _call(lib, "tsa_reset_device_status", FAKE + 4, None) == INVALID
     assert _call(lib, "tsa_get_device_status", None, None, None) == INVALID
+
+
+def test_per_head_budget_needs_head_counts(lib):
+    p = ctypes.byref(good(budget_mode="per_head"))
+    ws_n = T.stage_workspace_size(good(budget_mode="per_head"))
+    assert _call(lib, "tsa_budget", p, FAKE, None, FAKE, FAKE, ws_n, None) == INVALID
+    # the shared-budget modes accept a NULL k_head (scratch in the workspace)
+    p_max = ctypes.byref(good())
+    assert _call(lib, "tsa_budget", p_max, FAKE, None, FAKE, FAKE, 0, None) == WORKSPACE
 
 
 def test_workspace_missing_or_small(lib):

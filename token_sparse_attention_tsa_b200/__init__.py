@@ -24,6 +24,8 @@ STATUS_NAMES = {0: "TSA_OK", 1: "TSA_ERR_INVALID_ARG", 2: "TSA_ERR_UNSUPPORTED",
                 4: "TSA_ERR_CUDA", 5: "TSA_ERR_NONFINITE", 6: "TSA_ERR_TIMEOUT", 7: "TSA_ERR_BAD_INDEX"}
 DEVFLAG_NONFINITE, DEVFLAG_TIMEOUT, DEVFLAG_BAD_INDEX = 0x1, 0x2, 0x4
 FLAG_TEST_STALL = 0x80000000
+BUDGET_MAX, BUDGET_MEAN, BUDGET_PER_HEAD = 0, 1, 2
+BUDGET_MODES = {"max": BUDGET_MAX, "mean": BUDGET_MEAN, "per_head": BUDGET_PER_HEAD}
 
 # Every symbol the header declares (checked by the tests).
 EXPORTED = ("tsa_abi_version", "tsa_status_string", "tsa_check_params", "tsa_workspace_size",
@@ -42,11 +44,16 @@ class tsa_params(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
                 ("L", ctypes.c_int32), ("d", ctypes.c_int32), ("w", ctypes.c_int32),
                 ("tau", ctypes.c_float), ("softmax_scale", ctypes.c_float),
-                ("flags", ctypes.c_uint32), ("timeout_ms", ctypes.c_uint32)]
+                ("flags", ctypes.c_uint32), ("timeout_ms", ctypes.c_uint32),
+                ("budget_mode", ctypes.c_int32), ("keep_recent", ctypes.c_int32)]
 
 
-def params(B, Hq, Hkv, L, d, w, tau, softmax_scale=0.0, timeout_ms=0, flags=0) -> tsa_params:
-    return tsa_params(B, Hq, Hkv, L, d, w, tau, softmax_scale, flags, timeout_ms)
+def params(B, Hq, Hkv, L, d, w, tau, softmax_scale=0.0, timeout_ms=0, flags=0, budget_mode=BUDGET_MAX,
+           keep_recent=0) -> tsa_params:
+    """budget_mode: BUDGET_MAX / BUDGET_MEAN / BUDGET_PER_HEAD or "max" / "mean" / "per_head"."""
+    if isinstance(budget_mode, str):
+        budget_mode = BUDGET_MODES[budget_mode]
+    return tsa_params(B, Hq, Hkv, L, d, w, tau, softmax_scale, flags, timeout_ms, budget_mode, keep_recent)
 
 
 _lock = threading.Lock()
@@ -268,13 +275,15 @@ def tsa_forward(p, q, k, v, o, ws, scores_out=None, idx_out=None, k_seq_out=None
                               _ptr(ws, "ws"), _nbytes(ws), _stream(stream)), "tsa_forward")
 
 
-def forward(q, k, v, w: int, tau: float, softmax_scale: float = 0.0, ws=None, return_intermediates=False):
+def forward(q, k, v, w: int, tau: float, softmax_scale: float = 0.0, ws=None, return_intermediates=False,
+            budget_mode=BUDGET_MAX, keep_recent: int = 0):
     """Convenience wrapper: allocate the output (and workspace if not given)
-    and run ``tsa_forward`` on the current stream."""
+    and run ``tsa_forward`` on the current stream.  With intermediates, the
+    kept counts come back as [B], or [B, Hq] in the per-head budget mode."""
     import torch
     B, Hq, L, d = q.shape
     Hkv = k.shape[1]
-    p = params(B, Hq, Hkv, L, d, w, tau, softmax_scale)
+    p = params(B, Hq, Hkv, L, d, w, tau, softmax_scale, budget_mode=budget_mode, keep_recent=keep_recent)
     if ws is None:
         ws = new_workspace(p, full=True, device=q.device)
     o = torch.empty_like(q)
@@ -283,6 +292,7 @@ def forward(q, k, v, w: int, tau: float, softmax_scale: float = 0.0, ws=None, re
         return o
     scores = torch.empty((B, Hq, L), dtype=torch.float32, device=q.device)
     idx = torch.empty((B, Hq, L), dtype=torch.int32, device=q.device)
-    k_seq = torch.empty((B,), dtype=torch.int32, device=q.device)
+    kshape = (B, Hq) if p.budget_mode == BUDGET_PER_HEAD else (B,)
+    k_seq = torch.empty(kshape, dtype=torch.int32, device=q.device)
     tsa_forward(p, q, k, v, o, ws, scores, idx, k_seq)
     return o, scores, idx, k_seq

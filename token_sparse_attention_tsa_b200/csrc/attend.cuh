@@ -24,7 +24,7 @@
 namespace tsa {
 
 struct AttnArgs {
-  const int32_t* k_seq;   // valid rows per sequence (null: L)
+  Kept kept;              // valid rows per (b, h) (null counts: L)
   __nv_bfloat16* o;       // [B*Hq, L, D]
   float* lse;             // [B*Hq, L] or null
   uint32_t* status;       // device status word or null
@@ -120,8 +120,7 @@ __global__ void __launch_bounds__(Attn2Layout<D>::THREADS, 1)
   const int n_pairs = (a.n_tiles + 1) >> 1;
   const int t0 = 2 * (n_pairs - 1 - static_cast<int>(blockIdx.x));  // longest pairs first
 
-  int valid = a.k_seq ? a.k_seq[b] : a.L;
-  valid = valid < 0 ? 0 : (valid > a.L ? a.L : valid);
+  const int valid = a.kept.of(b, h, a.L);
   if (t0 * C::BM >= valid) return;                 // uniform, before any barrier
   const bool two = (t0 + 1) * C::BM < valid;       // second query tile has rows
   const int last0 = t0;                            // tile 0 attends KV tiles 0..t0

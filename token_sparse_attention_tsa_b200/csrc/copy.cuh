@@ -15,12 +15,14 @@
 
 #include <cuda_bf16.h>
 
+#include "sm100.cuh"
+
 namespace tsa {
 
 struct GatherArgs {
   const __nv_bfloat16 *q, *k, *v;  // [B*Hq, L, D], [B*Hkv, L, D] x2
   const int32_t* idx;              // [B*Hq, L]
-  const int32_t* k_seq;            // [B]
+  Kept kept;                       // rows kept per (b, h)
   __nv_bfloat16 *qc, *kc, *vc;     // [B*Hq, L, D]; qc may be null (K and V only)
   uint32_t* status;                // or null
   int L, Hq, Hkv, G;
@@ -39,8 +41,7 @@ __global__ void __launch_bounds__(256) gather_kernel(const GatherArgs a) {
     const int i = static_cast<int>(row - bh * a.L);
     const int b = static_cast<int>(bh / a.Hq);
     const int h = static_cast<int>(bh - static_cast<long long>(b) * a.Hq);
-    const int kb = __ldg(a.k_seq + b);
-    if (i >= kb) continue;
+    if (i >= a.kept.of(b, h, a.L)) continue;
     const int j = __ldg(a.idx + row);
     const size_t dst = static_cast<size_t>(row) * D + sub * 8;
     if (j < 0 || j >= a.L) {
@@ -65,7 +66,7 @@ __global__ void __launch_bounds__(256) gather_kernel(const GatherArgs a) {
 struct ScatterArgs {
   const __nv_bfloat16* oc;  // [B*Hq, L, D]
   const int32_t* idx;       // [B*Hq, L]
-  const int32_t* k_seq;     // [B]
+  Kept kept;                // rows kept per (b, h)
   __nv_bfloat16* o;         // [B*Hq, L, D]
   uint32_t* status;         // or null
   int L, Hq;
@@ -86,8 +87,7 @@ __global__ void __launch_bounds__(256) scatter_kernel(const ScatterArgs a) {
   const int bh = blockIdx.y;
   const int r0 = blockIdx.x * SCAT_ROWS;
   const int b = bh / a.Hq;
-  int kb = __ldg(a.k_seq + b);
-  kb = kb < 0 ? 0 : (kb > a.L ? a.L : kb);
+  const int kb = a.kept.of(b, bh - b * a.Hq, a.L);
   const int32_t* ix = a.idx + static_cast<size_t>(bh) * a.L;
   where[threadIdx.x] = -1;
   if (threadIdx.x == 0) {  // first i with ix[i] >= r0

@@ -12,7 +12,11 @@
 //         product is exact in fp64 and ceil is exact),
 //   T     = floor(tau * (double)sum_j q_j) (one fp64 multiply),
 //   p_h   = the largest count of least-important tokens whose masses sum to
-//           <= T; k_head = L - p_h; k_seq[b] = max over the heads of b.
+//           <= T; k_head = max(L - p_h, r) with r the forced recent tokens;
+//   k_seq[b] = max over the heads of b, or the ceiling of their mean.
+// The page calls the budget global without saying how heads combine: the
+// maximum is the default reading; the mean and a per-head budget (every
+// head keeps its own k_head) are the two other plain readings, selectable.
 // Ascending order of q_j is the ascending order of the fp32 bit patterns, so
 // neither kernel sorts: both run a most-significant-digit radix descent
 // (4 levels of 8 bits) over the score bit patterns with per-warp shared
@@ -21,6 +25,8 @@
 #pragma once
 
 #include <cstdint>
+
+#include "sm100.cuh"
 
 namespace tsa {
 
@@ -94,10 +100,10 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* r
 
 struct BudgetArgs {
   const float* scores;  // [B*Hq, L]
-  int32_t* k_head;      // [B*Hq] or null
-  int32_t* k_seq;       // [B], zeroed before launch
+  int32_t* k_head;      // [B*Hq]
   uint32_t* status;     // or null
   int L, Hq;
+  int keep_recent;      // r in [0, L]: every k_head is raised to at least r
   double tau;           // fp32 tau widened
 };
 
@@ -189,18 +195,46 @@ __global__ void __launch_bounds__(BS_THREADS, 1) budget_kernel(const BudgetArgs 
       p += static_cast<uint32_t>(s_rem / qstar);
     }
     const int32_t kh = a.L - static_cast<int32_t>(p);
-    if (a.k_head) a.k_head[bh] = kh;
-    atomicMax(&a.k_seq[bh / a.Hq], kh);
+    a.k_head[bh] = kh > a.keep_recent ? kh : a.keep_recent;
   }
   if (a.status && __syncthreads_or(bad) && threadIdx.x == 0) atomicOr(a.status, 0x1u);
 }
 
+// k_seq[b] from the heads' counts: mode 1 the ceiling of their mean, else
+// their maximum.  grid: B CTAs of 32 threads.
+__global__ void __launch_bounds__(32) budget_finalize_kernel(const int32_t* k_head, int32_t* k_seq, int Hq,
+                                                             int mode) {
+  const int b = blockIdx.x;
+  long long sum = 0;
+  int mx = 0;
+  for (int h = threadIdx.x; h < Hq; h += 32) {
+    const int k = k_head[static_cast<size_t>(b) * Hq + h];
+    sum += k;
+    mx = k > mx ? k : mx;
+  }
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) {
+    sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    const int y = __shfl_xor_sync(0xffffffffu, mx, o);
+    mx = y > mx ? y : mx;
+  }
+  if (threadIdx.x == 0) k_seq[b] = mode == 1 ? static_cast<int32_t>((sum + Hq - 1) / Hq) : mx;
+}
+
 struct SelectArgs {
   const float* scores;   // [B*Hq, L]
-  const int32_t* k_seq;  // [B]
+  Kept kept;             // rows kept per (b, h)
   int32_t* idx;          // [B*Hq, L]
   int L, Hq;
+  int keep_recent;       // tokens [L - r, L) rank above every score
 };
+
+// Selection key: the score's order key, or the top key for a forced token
+// (no score maps there: order keys of valid scores stay below 2^31).
+__device__ __forceinline__ uint32_t select_key(float s, int j, int first_forced, bool& bad) {
+  const uint32_t u = score_key(s, bad);
+  return j >= first_forced ? 0xffffffffu : u;
+}
 
 // grid: B*Hq CTAs of 1024 threads; dynamic smem: per-warp count histograms.
 __global__ void __launch_bounds__(BS_THREADS, 1) select_kernel(const SelectArgs a) {
@@ -213,8 +247,8 @@ __global__ void __launch_bounds__(BS_THREADS, 1) select_kernel(const SelectArgs 
   const int L = a.L;
   const float* sc = a.scores + static_cast<size_t>(bh) * L;
   int32_t* out = a.idx + static_cast<size_t>(bh) * L;
-  int k = a.k_seq[bh / a.Hq];
-  k = k < 0 ? 0 : (k > L ? L : k);
+  const int k = a.kept.of(bh / a.Hq, bh % a.Hq, L);
+  const int first_forced = L - a.keep_recent;
   const int warp = threadIdx.x >> 5;
   bool bad = false;
 
@@ -240,7 +274,7 @@ __global__ void __launch_bounds__(BS_THREADS, 1) select_kernel(const SelectArgs 
     __syncthreads();
     const uint32_t prefix = s_prefix, mask = s_mask;
     for (int j = threadIdx.x; j < L; j += BS_THREADS) {
-      const uint32_t u = score_key(sc[j], bad);
+      const uint32_t u = select_key(sc[j], j, first_forced, bad);
       if ((u & mask) == prefix) atomicAdd(&hcnt[warp * 256 + ((u >> shift) & 255u)], 1u);
     }
     __syncthreads();
@@ -276,7 +310,7 @@ __global__ void __launch_bounds__(BS_THREADS, 1) select_kernel(const SelectArgs 
   const int j1 = min(L, j0 + per);
   uint32_t gt = 0, eq = 0;
   for (int j = j0; j < j1; ++j) {
-    const uint32_t u = score_key(sc[j], bad);
+    const uint32_t u = select_key(sc[j], j, first_forced, bad);
     gt += (u > ut);
     eq += (u == ut);
   }
@@ -287,7 +321,7 @@ __global__ void __launch_bounds__(BS_THREADS, 1) select_kernel(const SelectArgs 
   uint32_t pos = block_exclusive_scan(gt + take_eq, red, cnt_total);
   uint32_t eq_seen = eq_before;
   for (int j = j0; j < j1; ++j) {
-    const uint32_t u = score_key(sc[j], bad);
+    const uint32_t u = select_key(sc[j], j, first_forced, bad);
     bool take = u > ut;
     if (u == ut) {
       take = eq_seen < need;

@@ -350,4 +350,17 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
+// Rows kept by each (sequence b, head h): n[b * sb + h * sh], clipped to
+// [0, L].  Per-sequence counts use (sb, sh) = (1, 0), per-head counts
+// (Hq, 1); a null n keeps every row (the dense case).
+struct Kept {
+  const int32_t* n;
+  int sb, sh;
+  __device__ __forceinline__ int of(int b, int h, int L) const {
+    if (!n) return L;
+    const int k = __ldg(n + static_cast<size_t>(b) * sb + static_cast<size_t>(h) * sh);
+    return k < 0 ? 0 : (k > L ? L : k);
+  }
+};
+
 }  // namespace tsa

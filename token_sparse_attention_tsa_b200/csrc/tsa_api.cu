@@ -36,12 +36,13 @@ int score_chunks(const tsa_params* p) {
   return (p->L + span - 1) / span;
 }
 
-// Workspace layout.  Stage part: status word (+ abort words), score scratch.
+// Workspace layout.  Stage part: status word (+ abort words), score scratch,
+// per-head budget scratch.
 // Forward part: scores, idx, k_head, k_seq and the compressed Q, K and V.
 // (tsa_forward's attention writes its output in place, so no compressed
 // output is stored.)
 struct WsLayout {
-  size_t status = 0, part_m = 0, part_z = 0, stats = 0, stage_end = 0;
+  size_t status = 0, part_m = 0, part_z = 0, stats = 0, kh_scratch = 0, stage_end = 0;
   size_t scores = 0, idx = 0, k_head = 0, k_seq = 0, qc = 0, kc = 0, vc = 0, total = 0;
 };
 
@@ -55,6 +56,7 @@ WsLayout layout_of(const tsa_params* p) {
   w.part_m = off;           off = align_up(off + rows * nch * sizeof(float));
   w.part_z = off;           off = align_up(off + rows * nch * sizeof(double));
   w.stats = off;            off = align_up(off + rows * sizeof(float2));
+  w.kh_scratch = off;       off = align_up(off + bhq * sizeof(int32_t));
   w.stage_end = off;
   const size_t tok = bhq * static_cast<size_t>(p->L);
   w.scores = off;           off = align_up(off + tok * sizeof(float));
@@ -71,6 +73,14 @@ WsLayout layout_of(const tsa_params* p) {
 template <typename T>
 T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+bool per_head(const tsa_params* p) { return p->budget_mode == TSA_BUDGET_PER_HEAD; }
+
+// Kept-row counts as the kernels read them: per sequence [B], or per head
+// [B, Hq] in the per-head budget mode.
+tsa::Kept kept_of(const tsa_params* p, const int32_t* n) {
+  return per_head(p) ? tsa::Kept{n, p->Hq, 1} : tsa::Kept{n, 1, 0};
 }
 
 float scale_of(const tsa_params* p) {
@@ -196,20 +206,24 @@ tsa_status run_score(const tsa_params* p, const void* q, const void* k, float* s
   return launch_ok();
 }
 
+// k_head receives every head's count (required); k_seq, when not null, the
+// per-sequence budget of the mode (max, or ceiling of the mean; per-head
+// mode reports the max).
 tsa_status run_budget(const tsa_params* p, const float* scores, int32_t* k_head, int32_t* k_seq,
                       uint32_t* status, cudaStream_t st) {
   if (!ensure_smem(g_budget, tsa::budget_kernel, kBudgetSmem)) return TSA_ERR_CUDA;
-  if (cudaMemsetAsync(k_seq, 0, sizeof(int32_t) * p->B, st) != cudaSuccess) return TSA_ERR_CUDA;
-  tsa::BudgetArgs a{scores, k_head, k_seq, status, p->L, p->Hq,
-                    static_cast<double>(p->tau)};
+  tsa::BudgetArgs a{scores, k_head, status, p->L, p->Hq, p->keep_recent, static_cast<double>(p->tau)};
   tsa::budget_kernel<<<p->B * p->Hq, tsa::BS_THREADS, kBudgetSmem, st>>>(a);
+  if (k_seq)
+    tsa::budget_finalize_kernel<<<p->B, 32, 0, st>>>(k_head, k_seq, p->Hq,
+                                                     p->budget_mode == TSA_BUDGET_MEAN ? 1 : 0);
   return launch_ok();
 }
 
-tsa_status run_select(const tsa_params* p, const float* scores, const int32_t* k_seq, int32_t* idx,
+tsa_status run_select(const tsa_params* p, const float* scores, const int32_t* kept, int32_t* idx,
                       cudaStream_t st) {
   if (!ensure_smem(g_select, tsa::select_kernel, kSelectSmem)) return TSA_ERR_CUDA;
-  tsa::SelectArgs a{scores, k_seq, idx, p->L, p->Hq};
+  tsa::SelectArgs a{scores, kept_of(p, kept), idx, p->L, p->Hq, p->keep_recent};
   tsa::select_kernel<<<p->B * p->Hq, tsa::BS_THREADS, kSelectSmem, st>>>(a);
   return launch_ok();
 }
@@ -227,7 +241,7 @@ tsa_status run_gather(const tsa_params* p, const void* q, const void* k, const v
   a.k = static_cast<const __nv_bfloat16*>(k);
   a.v = static_cast<const __nv_bfloat16*>(v);
   a.idx = idx;
-  a.k_seq = k_seq;
+  a.kept = kept_of(p, k_seq);
   a.qc = static_cast<__nv_bfloat16*>(qc);
   a.kc = static_cast<__nv_bfloat16*>(kc);
   a.vc = static_cast<__nv_bfloat16*>(vc);
@@ -246,8 +260,8 @@ tsa_status run_gather(const tsa_params* p, const void* q, const void* k, const v
 
 tsa_status run_scatter(const tsa_params* p, const void* oc, const int32_t* idx, const int32_t* k_seq, void* o,
                        uint32_t* status, cudaStream_t st) {
-  tsa::ScatterArgs a{static_cast<const __nv_bfloat16*>(oc), idx, k_seq, static_cast<__nv_bfloat16*>(o),
-                     status, p->L, p->Hq};
+  tsa::ScatterArgs a{static_cast<const __nv_bfloat16*>(oc), idx, kept_of(p, k_seq),
+                     static_cast<__nv_bfloat16*>(o), status, p->L, p->Hq};
   const dim3 g((p->L + tsa::SCAT_ROWS - 1) / tsa::SCAT_ROWS, p->B * p->Hq);
   if (p->d == 128)
     tsa::scatter_kernel<128><<<g, 256, 0, st>>>(a);
@@ -282,7 +296,7 @@ tsa_status run_attend(const tsa_params* p, const void* q, const void* k, const v
   if (!maps_ok) return TSA_ERR_CUDA;
   if (cudaMemsetAsync(abort_word, 0, sizeof(uint32_t), st) != cudaSuccess) return TSA_ERR_CUDA;
   tsa::AttnArgs a;
-  a.k_seq = k_seq;
+  a.kept = kept_of(p, k_seq);
   a.o = static_cast<__nv_bfloat16*>(o);
   a.lse = lse;
   a.status = status;
@@ -318,7 +332,7 @@ tsa_status run_attend(const tsa_params* p, const void* q, const void* k, const v
 // they are).
 tsa_status run_zero_unselected(const tsa_params* p, const int32_t* idx, const int32_t* k_seq, void* o,
                                uint32_t* status, cudaStream_t st) {
-  tsa::ScatterArgs a{nullptr, idx, k_seq, static_cast<__nv_bfloat16*>(o), status, p->L, p->Hq};
+  tsa::ScatterArgs a{nullptr, idx, kept_of(p, k_seq), static_cast<__nv_bfloat16*>(o), status, p->L, p->Hq};
   const dim3 g((p->L + tsa::SCAT_ROWS - 1) / tsa::SCAT_ROWS, p->B * p->Hq);
   if (p->d == 128)
     tsa::scatter_kernel<128, true><<<g, 256, 0, st>>>(a);
@@ -372,6 +386,8 @@ tsa_status tsa_check_params(const tsa_params* p) {
   if (!(p->tau >= 0.f && p->tau < 1.f)) return TSA_ERR_INVALID_ARG;
   if (!(p->softmax_scale >= 0.f) || std::isinf(p->softmax_scale)) return TSA_ERR_INVALID_ARG;
   if ((p->flags & ~TSA_FLAG_TEST_STALL) != 0) return TSA_ERR_INVALID_ARG;
+  if (p->budget_mode < TSA_BUDGET_MAX || p->budget_mode > TSA_BUDGET_PER_HEAD) return TSA_ERR_INVALID_ARG;
+  if (p->keep_recent < 0 || p->keep_recent > p->L) return TSA_ERR_INVALID_ARG;
   if (p->d != 64 && p->d != 128) return TSA_ERR_UNSUPPORTED;
   if (p->w > 4096 || p->L > (1 << 22)) return TSA_ERR_UNSUPPORTED;
   if (static_cast<long long>(p->B) * p->Hq * p->L >= (1LL << 31)) return TSA_ERR_UNSUPPORTED;
@@ -426,8 +442,10 @@ tsa_status tsa_budget(const tsa_params* p, const float* scores, int32_t* k_head,
   tsa_status s = tsa_check_params(p);
   if (s != TSA_OK) return s;
   if (!tensors_ok({scores, k_seq}) || (k_head && !aligned(k_head, 4))) return TSA_ERR_INVALID_ARG;
+  if (per_head(p) && !k_head) return TSA_ERR_INVALID_ARG;  // the per-head counts are the budget
   if ((s = check_ws(p, ws, ws_bytes, false)) != TSA_OK) return s;
-  return run_budget(p, scores, k_head, k_seq, status_of(ws), static_cast<cudaStream_t>(stream));
+  int32_t* kh = k_head ? k_head : at<int32_t>(ws, layout_of(p).kh_scratch);
+  return run_budget(p, scores, kh, k_seq, status_of(ws), static_cast<cudaStream_t>(stream));
 }
 
 tsa_status tsa_select(const tsa_params* p, const float* scores, const int32_t* k_seq, int32_t* idx, void* ws,
@@ -492,9 +510,12 @@ tsa_status tsa_forward(const tsa_params* p, const void* q, const void* k, const 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   float* scores = scores_out ? scores_out : at<float>(ws, w.scores);
   int32_t* idx = idx_out ? idx_out : at<int32_t>(ws, w.idx);
-  int32_t* kseq = k_seq_out ? k_seq_out : at<int32_t>(ws, w.k_seq);
+  // kept counts: k_seq [B] (max / mean), or the heads' own counts [B, Hq]
+  int32_t* khead = (per_head(p) && k_seq_out) ? k_seq_out : at<int32_t>(ws, w.k_head);
+  int32_t* kbud = (!per_head(p) && k_seq_out) ? k_seq_out : at<int32_t>(ws, w.k_seq);
+  int32_t* kseq = per_head(p) ? khead : kbud;
   if ((s = run_score(p, q, k, scores, ws, st)) != TSA_OK) return s;
-  if ((s = run_budget(p, scores, at<int32_t>(ws, w.k_head), kseq, status_of(ws), st)) != TSA_OK) return s;
+  if ((s = run_budget(p, scores, khead, kbud, status_of(ws), st)) != TSA_OK) return s;
   if ((s = run_select(p, scores, kseq, idx, st)) != TSA_OK) return s;
   // gather once, attention writing each output row in place, zeros for the
   // unselected rows (tsa_gather_qkv + tsa_attend_scatter)
