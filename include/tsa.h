@@ -20,7 +20,13 @@
  *
  * Layouts (all row-major, contiguous, little-endian):
  *   q        bf16 [B, Hq,  L, d]      k, v   bf16 [B, Hkv, L, d]
- *   o        bf16 [B, Hq,  L, d]      scores fp32 [B, Hq, L]
+ *   o        bf16 [B, Hq,  L, d]
+ *            (head-major, p->layout == TSA_LAYOUT_BHLD, the default), or
+ *            token-major with p->layout == TSA_LAYOUT_BLHD: q, o
+ *            [B, L, Hq, d] and k, v [B, L, Hkv, d], the layout a prefill
+ *            engine's projections produce.  Only the caller's q, k, v, o
+ *            follow p->layout; every tensor below is always head-major.
+ *   scores   fp32 [B, Hq, L]
  *   idx      int32 [B, Hq, L]: entries [0, k_b) hold S_h ascending, the rest -1
  *   k_head   int32 [B, Hq]            k_seq  int32 [B]
  *   kept     the rows kept by every head, argument of the calls after the
@@ -89,6 +95,10 @@ typedef enum tsa_status {
  * heads combine; MAX (every head of sequence b keeps k_b = max_h k_head) is
  * the default reading, MEAN (k_b = ceil(mean_h k_head)) and PER_HEAD (head h
  * keeps its own k_head, no shared budget) are the two other plain ones. */
+/* tsa_params.layout: memory order of the caller's q, k, v and o. */
+#define TSA_LAYOUT_BHLD 0
+#define TSA_LAYOUT_BLHD 1
+
 #define TSA_BUDGET_MAX 0
 #define TSA_BUDGET_MEAN 1
 #define TSA_BUDGET_PER_HEAD 2
@@ -109,6 +119,7 @@ typedef struct tsa_params {
   int32_t keep_recent;  /* 0 <= r <= L: the last r tokens of every sequence
                            are kept in every head (each k_head is raised to
                            at least r; the selection ranks them first)       */
+  int32_t layout;       /* TSA_LAYOUT_BHLD (0) or TSA_LAYOUT_BLHD (1)        */
 } tsa_params;
 
 /* Version of this ABI (TSA_ABI_VERSION of the built library). */

@@ -63,6 +63,7 @@ def test_status_strings(lib):
     (dict(budget_mode=-1), INVALID), (dict(budget_mode=3), INVALID), (dict(budget_mode="mean"), 0),
     (dict(budget_mode="per_head"), 0), (dict(keep_recent=-1), INVALID), (dict(keep_recent=4097), INVALID),
     (dict(keep_recent=4096), 0), (dict(keep_recent=64, budget_mode="per_head"), 0),
+    (dict(layout="blhd"), 0), (dict(layout=2), INVALID), (dict(layout=-1), INVALID),
 ])
 def test_param_validation(lib, kw, want):
     p = good(**kw)

@@ -26,6 +26,8 @@ DEVFLAG_NONFINITE, DEVFLAG_TIMEOUT, DEVFLAG_BAD_INDEX = 0x1, 0x2, 0x4
 FLAG_TEST_STALL = 0x80000000
 BUDGET_MAX, BUDGET_MEAN, BUDGET_PER_HEAD = 0, 1, 2
 BUDGET_MODES = {"max": BUDGET_MAX, "mean": BUDGET_MEAN, "per_head": BUDGET_PER_HEAD}
+LAYOUT_BHLD, LAYOUT_BLHD = 0, 1
+LAYOUTS = {"bhld": LAYOUT_BHLD, "blhd": LAYOUT_BLHD}
 
 # Every symbol the header declares (checked by the tests).
 EXPORTED = ("tsa_abi_version", "tsa_status_string", "tsa_check_params", "tsa_workspace_size",
@@ -45,15 +47,18 @@ class tsa_params(ctypes.Structure):
                 ("L", ctypes.c_int32), ("d", ctypes.c_int32), ("w", ctypes.c_int32),
                 ("tau", ctypes.c_float), ("softmax_scale", ctypes.c_float),
                 ("flags", ctypes.c_uint32), ("timeout_ms", ctypes.c_uint32),
-                ("budget_mode", ctypes.c_int32), ("keep_recent", ctypes.c_int32)]
+                ("budget_mode", ctypes.c_int32), ("keep_recent", ctypes.c_int32), ("layout", ctypes.c_int32)]
 
 
 def params(B, Hq, Hkv, L, d, w, tau, softmax_scale=0.0, timeout_ms=0, flags=0, budget_mode=BUDGET_MAX,
-           keep_recent=0) -> tsa_params:
-    """budget_mode: BUDGET_MAX / BUDGET_MEAN / BUDGET_PER_HEAD or "max" / "mean" / "per_head"."""
+           keep_recent=0, layout=LAYOUT_BHLD) -> tsa_params:
+    """budget_mode: BUDGET_MAX / BUDGET_MEAN / BUDGET_PER_HEAD or "max" / "mean" / "per_head".
+    layout: LAYOUT_BHLD / LAYOUT_BLHD or "bhld" / "blhd" (memory order of q, k, v, o)."""
     if isinstance(budget_mode, str):
         budget_mode = BUDGET_MODES[budget_mode]
-    return tsa_params(B, Hq, Hkv, L, d, w, tau, softmax_scale, flags, timeout_ms, budget_mode, keep_recent)
+    if isinstance(layout, str):
+        layout = LAYOUTS[layout]
+    return tsa_params(B, Hq, Hkv, L, d, w, tau, softmax_scale, flags, timeout_ms, budget_mode, keep_recent, layout)
 
 
 _lock = threading.Lock()
@@ -276,14 +281,23 @@ def tsa_forward(p, q, k, v, o, ws, scores_out=None, idx_out=None, k_seq_out=None
 
 
 def forward(q, k, v, w: int, tau: float, softmax_scale: float = 0.0, ws=None, return_intermediates=False,
-            budget_mode=BUDGET_MAX, keep_recent: int = 0):
+            budget_mode=BUDGET_MAX, keep_recent: int = 0, layout="bhld"):
     """Convenience wrapper: allocate the output (and workspace if not given)
-    and run ``tsa_forward`` on the current stream.  With intermediates, the
-    kept counts come back as [B], or [B, Hq] in the per-head budget mode."""
+    and run ``tsa_forward`` on the current stream.  q, k, v are [B, H, L, d]
+    (layout "bhld") or [B, L, H, d] ("blhd"); o comes back in the same
+    layout.  With intermediates, the kept counts come back as [B], or
+    [B, Hq] in the per-head budget mode."""
     import torch
-    B, Hq, L, d = q.shape
-    Hkv = k.shape[1]
-    p = params(B, Hq, Hkv, L, d, w, tau, softmax_scale, budget_mode=budget_mode, keep_recent=keep_recent)
+    if isinstance(layout, str):
+        layout = LAYOUTS[layout]
+    if layout == LAYOUT_BLHD:
+        B, L, Hq, d = q.shape
+        Hkv = k.shape[2]
+    else:
+        B, Hq, L, d = q.shape
+        Hkv = k.shape[1]
+    p = params(B, Hq, Hkv, L, d, w, tau, softmax_scale, budget_mode=budget_mode, keep_recent=keep_recent,
+               layout=layout)
     if ws is None:
         ws = new_workspace(p, full=True, device=q.device)
     o = torch.empty_like(q)

@@ -25,7 +25,8 @@ namespace tsa {
 
 struct AttnArgs {
   Kept kept;              // valid rows per (b, h) (null counts: L)
-  __nv_bfloat16* o;       // [B*Hq, L, D]
+  __nv_bfloat16* o;       // B x Hq heads of L rows of D
+  RowStrides os;          // row strides of o
   float* lse;             // [B*Hq, L] or null
   uint32_t* status;       // device status word or null
   uint32_t* abort_word;   // launch-wide abort word (zeroed before launch) or null
@@ -38,6 +39,7 @@ struct AttnArgs {
   float scale_log2;       // softmax scale * log2(e)
   uint64_t limit_ns;      // per-wait time limit
   int test_stall;         // failure-path test: the MMA issuer first waits on a barrier nothing completes
+  int token_major;        // Q/K/V maps are (d, H, L, B) (else (d, L, H, B)); gather rows likewise
 };
 
 // ---------------------------------------------------------------------------
@@ -169,23 +171,27 @@ __global__ void __launch_bounds__(Attn2Layout<D>::THREADS, 1)
         tma_prefetch_desc(&tmK);
         tma_prefetch_desc(&tmV);
       }
-      const int zkv = b * a.Hkv_map + h / a.G_map;
-      // One 128-row tile into dst: a box load, or 32 four-row gathers whose
-      // row numbers come from idx (lane l reads entries 4l..4l+3; rows past
-      // the selection read row 0 of the head, masked or zeroed downstream).
-      auto load_tile = [&](auto by_index, uint32_t dst, const CUtensorMap* m, uint32_t br, int tile, int z) {
+      const bool tm = a.token_major != 0;
+      // One 128-row tile of head hz (of the map's nh heads) of sequence b
+      // into dst: a box load, or 32 four-row gathers whose row numbers come
+      // from idx (lane l reads entries 4l..4l+3; rows past the selection read
+      // token 0 of the head, masked or zeroed downstream).
+      auto load_tile = [&](auto by_index, uint32_t dst, const CUtensorMap* m, uint32_t br, int tile, int hz,
+                           int nh) {
         if constexpr (!decltype(by_index)::value) {
           if (leader) {
 #pragma unroll
-            for (int c = 0; c < C::NCH; ++c) tma_load_3d(dst + c * C::CHUNK, m, br, c * 64, tile * C::BM, z);
+            for (int c = 0; c < C::NCH; ++c)
+              tma_load_rows(dst + c * C::CHUNK, m, br, tm, c * 64, tile * C::BM, hz, b);
           }
         } else {
           int rr[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             const int i = tile * C::BM + 4 * lane + u;
-            const int v = i < valid ? __ldg(a.idx + static_cast<size_t>(bh) * a.L + i) : 0;
-            rr[u] = z * a.L + (v >= 0 && v < a.L ? v : 0);
+            int v = i < valid ? __ldg(a.idx + static_cast<size_t>(bh) * a.L + i) : 0;
+            v = (v >= 0 && v < a.L) ? v : 0;
+            rr[u] = tm ? (b * a.L + v) * nh + hz : (b * nh + hz) * a.L + v;
           }
 #pragma unroll 4
           for (int g = 0; g < 32; ++g) {
@@ -202,15 +208,16 @@ __global__ void __launch_bounds__(Attn2Layout<D>::THREADS, 1)
       __syncwarp();
       constexpr std::integral_constant<bool, kGather> q_by_index{};
       constexpr std::integral_constant<bool, kGather> kv_by_index{};
-      load_tile(q_by_index, base + C::OFF_Q0, &tmQ, bar(C::B_Q), t0, bh);
-      if (two) load_tile(q_by_index, base + C::OFF_Q1, &tmQ, bar(C::B_Q), t0 + 1, bh);
+      load_tile(q_by_index, base + C::OFF_Q0, &tmQ, bar(C::B_Q), t0, h, a.Hq);
+      if (two) load_tile(q_by_index, base + C::OFF_Q1, &tmQ, bar(C::B_Q), t0 + 1, h, a.Hq);
       int issued = 0;
       for (int n = 0; n < 2 * n_kv; ++n) {
         const int s = slot_of(n), u = use_of(n);
         if (u >= 1 && !__all_sync(0xffffffffu, mbar_wait(bar(C::B_EMPTY + s), (u - 1) & 1, wc))) break;
         if (leader) mbar_arrive_expect_tx(bar(C::B_FULL + s), C::TILE);
         __syncwarp();
-        load_tile(kv_by_index, ring(n), (n & 1) ? &tmV : &tmK, bar(C::B_FULL + s), n >> 1, zkv);
+        load_tile(kv_by_index, ring(n), (n & 1) ? &tmV : &tmK, bar(C::B_FULL + s), n >> 1, h / a.G_map,
+                  a.Hkv_map);
         issued = n + 1;
       }
       if (leader && *cta_abort) {  // let every copy still in flight land before exit
@@ -437,7 +444,7 @@ __global__ void __launch_bounds__(Attn2Layout<D>::THREADS, 1)
           if (a.status) atomicOr(a.status, 0x4u);
         }
       }
-      __nv_bfloat16* orow = a.o + (static_cast<size_t>(bh) * a.L + (store ? orow_index : 0)) * D;
+      __nv_bfloat16* orow = a.o + a.os.at(b, h, store ? orow_index : 0);
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         float ov[32];

@@ -20,7 +20,8 @@
 namespace tsa {
 
 struct GatherArgs {
-  const __nv_bfloat16 *q, *k, *v;  // [B*Hq, L, D], [B*Hkv, L, D] x2
+  const __nv_bfloat16 *q, *k, *v;  // q: B x Hq heads, k, v: B x Hkv heads of L rows of D
+  RowStrides qs, kvs;              // their row strides (head-major or token-major)
   const int32_t* idx;              // [B*Hq, L]
   Kept kept;                       // rows kept per (b, h)
   __nv_bfloat16 *qc, *kc, *vc;     // [B*Hq, L, D]; qc may be null (K and V only)
@@ -52,8 +53,8 @@ __global__ void __launch_bounds__(256) gather_kernel(const GatherArgs a) {
       *reinterpret_cast<uint4*>(a.vc + dst) = z;
       continue;
     }
-    const size_t sq = (static_cast<size_t>(bh) * a.L + j) * D + sub * 8;
-    const size_t skv = ((static_cast<size_t>(b) * a.Hkv + h / a.G) * a.L + j) * D + sub * 8;
+    const size_t sq = a.qs.at(b, h, j) + sub * 8;
+    const size_t skv = a.kvs.at(b, h / a.G, j) + sub * 8;
     const uint4 vk = __ldg(reinterpret_cast<const uint4*>(a.k + skv));
     const uint4 vv = __ldg(reinterpret_cast<const uint4*>(a.v + skv));
     if (a.qc) *reinterpret_cast<uint4*>(a.qc + dst) = __ldg(reinterpret_cast<const uint4*>(a.q + sq));
@@ -64,10 +65,11 @@ __global__ void __launch_bounds__(256) gather_kernel(const GatherArgs a) {
 }
 
 struct ScatterArgs {
-  const __nv_bfloat16* oc;  // [B*Hq, L, D]
+  const __nv_bfloat16* oc;  // [B*Hq, L, D] compressed (head-major)
   const int32_t* idx;       // [B*Hq, L]
   Kept kept;                // rows kept per (b, h)
-  __nv_bfloat16* o;         // [B*Hq, L, D]
+  __nv_bfloat16* o;         // B x Hq heads of L rows of D
+  RowStrides os;            // row strides of o (head-major or token-major)
   uint32_t* status;         // or null
   int L, Hq;
 };
@@ -119,7 +121,7 @@ __global__ void __launch_bounds__(256) scatter_kernel(const ScatterArgs a) {
     uint4 val = make_uint4(0, 0, 0, 0);
     if (!kZeroOnly && i >= 0)
       val = __ldg(reinterpret_cast<const uint4*>(a.oc + (static_cast<size_t>(bh) * a.L + i) * D + sub * 8));
-    __stcs(reinterpret_cast<uint4*>(a.o + (static_cast<size_t>(bh) * a.L + r) * D + sub * 8), val);
+    __stcs(reinterpret_cast<uint4*>(a.o + a.os.at(b, bh - b * a.Hq, r) + sub * 8), val);
   }
   if (bad && a.status) atomicOr(a.status, 0x4u);
 }

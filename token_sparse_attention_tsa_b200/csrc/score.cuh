@@ -48,6 +48,7 @@ struct ScoreArgs {
   int n_rb;                // window row blocks of 128
   float scale_log2;        // scale * log2(e)
   uint64_t limit_ns;
+  int token_major;         // q, k maps are (d, H, L, B) (else (d, L, H, B))
 };
 
 template <int D>
@@ -104,7 +105,6 @@ __global__ void __launch_bounds__(SC_THREADS, 1)
   const int chunk = blockIdx.x;
   const int bh = blockIdx.y;
   const int b = bh / a.Hq, h = bh - (bh / a.Hq) * a.Hq;
-  const int zkv = b * a.Hkv + h / a.G;
   const int key0 = chunk * SC_CHUNK_TILES * SC_KEYS;
   int n_kt = (a.L - key0 + SC_KEYS - 1) / SC_KEYS;
   n_kt = n_kt > SC_CHUNK_TILES ? SC_CHUNK_TILES : n_kt;
@@ -155,8 +155,9 @@ __global__ void __launch_bounds__(SC_THREADS, 1)
         const int krow = key0 + step_kt(s) * SC_KEYS;
 #pragma unroll
         for (int c = 0; c < C::NCH; ++c) {
-          tma_load_3d(sb + c * C::CHUNK, &tmQ, bar(SB_FULL + st), c * 64, qrow, bh);
-          tma_load_3d(sb + C::Q_BYTES + c * C::K_CHUNK, &tmK, bar(SB_FULL + st), c * 64, krow, zkv);
+          tma_load_rows(sb + c * C::CHUNK, &tmQ, bar(SB_FULL + st), a.token_major, c * 64, qrow, h, b);
+          tma_load_rows(sb + C::Q_BYTES + c * C::K_CHUNK, &tmK, bar(SB_FULL + st), a.token_major, c * 64, krow,
+                        h / a.G, b);
         }
       }
       issued = s + 1;

@@ -109,6 +109,26 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* m, 
       : "memory");
 }
 
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const CUtensorMap* m, uint32_t bar, int x, int y,
+                                            int z, int w) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(x), "r"(y), "r"(z), "r"(w)
+      : "memory");
+}
+
+// Token rows of a [B, H, L, d] (head-major) or [B, L, H, d] (token-major)
+// tensor seen through a 4D tensor map whose dimensions are (d, L, H, B) or
+// (d, H, L, B): the box at column x, token t, head h, sequence b.
+__device__ __forceinline__ void tma_load_rows(uint32_t dst, const CUtensorMap* m, uint32_t bar, bool token_major,
+                                              int x, int t, int h, int b) {
+  if (token_major)
+    tma_load_4d(dst, m, bar, x, h, t, b);
+  else
+    tma_load_4d(dst, m, bar, x, t, h, b);
+}
+
 // Generic-proxy shared-memory writes -> visible to the async proxy (TMA, MMA).
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -349,6 +369,16 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
   return d;
 }
+
+// Element offset of row (sequence b, head h, token t) of a bf16 tensor with
+// element strides sb, sh, st (head-major [B, H, L, d]: H*L*d, L*d, d;
+// token-major [B, L, H, d]: L*H*d, d, H*d).
+struct RowStrides {
+  long long sb, sh, st;
+  __device__ __forceinline__ size_t at(int b, int h, int t) const {
+    return static_cast<size_t>(b * sb + h * sh + t * st);
+  }
+};
 
 // Rows kept by each (sequence b, head h): n[b * sb + h * sh], clipped to
 // [0, L].  Per-sequence counts use (sb, sh) = (1, 0), per-head counts

@@ -77,6 +77,15 @@ T* at(void* ws, size_t off) {
 
 bool per_head(const tsa_params* p) { return p->budget_mode == TSA_BUDGET_PER_HEAD; }
 
+// The caller's q, k, v, o are token-major [B, L, H, d] (else head-major
+// [B, H, L, d]); compressed buffers, scores and indices are always head-major.
+bool token_major(const tsa_params* p) { return p->layout == TSA_LAYOUT_BLHD; }
+
+tsa::RowStrides strides_of(bool tm, int heads, int L, int d) {
+  const long long H = heads, Ll = L, dd = d;
+  return tm ? tsa::RowStrides{Ll * H * dd, dd, H * dd} : tsa::RowStrides{H * Ll * dd, Ll * dd, dd};
+}
+
 // Kept-row counts as the kernels read them: per sequence [B], or per head
 // [B, Hq] in the per-head budget mode.
 tsa::Kept kept_of(const tsa_params* p, const int32_t* n) {
@@ -111,15 +120,21 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// [heads, L, d] bf16 rows; box = box_rows rows x 64 columns, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, int d, int L, int heads, int box_rows = 128) {
+// bf16 rows of B sequences x `heads` heads x L tokens x d: dimensions
+// (d, L, heads, B) for head-major memory, (d, heads, L, B) for token-major
+// (strides ascend either way); box = box_rows tokens x 64 columns of one
+// head, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, int d, int L, int heads, int B, bool tm, int box_rows = 128) {
   auto fn = encode_fn();
   if (!fn) return false;
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(L), static_cast<cuuint64_t>(heads)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2, static_cast<cuuint64_t>(L) * d * 2};
-  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+  const cuuint64_t D = static_cast<cuuint64_t>(d), Ll = static_cast<cuuint64_t>(L),
+                   H = static_cast<cuuint64_t>(heads), Bb = static_cast<cuuint64_t>(B);
+  cuuint64_t dims[4] = {D, tm ? H : Ll, tm ? Ll : H, Bb};
+  cuuint64_t strides[3] = {D * 2, D * 2 * dims[1], D * 2 * dims[1] * dims[2]};
+  const cuuint32_t rows = static_cast<cuuint32_t>(box_rows);
+  cuuint32_t box[4] = {64, tm ? 1u : rows, tm ? rows : 1u, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -164,8 +179,9 @@ tsa_status run_score(const tsa_params* p, const void* q, const void* k, float* s
   const WsLayout w = layout_of(p);
   const int bhq = p->B * p->Hq;
   CUtensorMap mq, mk;
-  if (!make_map(&mq, q, p->d, p->L, bhq, tsa::SC_ROWS) ||
-      !make_map(&mk, k, p->d, p->L, p->B * p->Hkv, tsa::SC_KEYS))
+  const bool tm = token_major(p);
+  if (!make_map(&mq, q, p->d, p->L, p->Hq, p->B, tm, tsa::SC_ROWS) ||
+      !make_map(&mk, k, p->d, p->L, p->Hkv, p->B, tm, tsa::SC_KEYS))
     return TSA_ERR_CUDA;
   tsa::ScoreArgs a;
   a.scores = scores;
@@ -183,6 +199,7 @@ tsa_status run_score(const tsa_params* p, const void* q, const void* k, float* s
   a.n_rb = (p->w + tsa::SC_ROWS - 1) / tsa::SC_ROWS;
   a.scale_log2 = scale_of(p) * 1.4426950408889634f;
   a.limit_ns = limit_ns_of(p);
+  a.token_major = tm ? 1 : 0;
   const dim3 grid(a.n_chunks, bhq);
   const int rows = bhq * p->w;
   if (cudaMemsetAsync(a.abort_word, 0, sizeof(uint32_t), st) != cudaSuccess) return TSA_ERR_CUDA;
@@ -242,6 +259,8 @@ tsa_status run_gather(const tsa_params* p, const void* q, const void* k, const v
   a.v = static_cast<const __nv_bfloat16*>(v);
   a.idx = idx;
   a.kept = kept_of(p, k_seq);
+  a.qs = strides_of(token_major(p), p->Hq, p->L, p->d);
+  a.kvs = strides_of(token_major(p), p->Hkv, p->L, p->d);
   a.qc = static_cast<__nv_bfloat16*>(qc);
   a.kc = static_cast<__nv_bfloat16*>(kc);
   a.vc = static_cast<__nv_bfloat16*>(vc);
@@ -261,7 +280,8 @@ tsa_status run_gather(const tsa_params* p, const void* q, const void* k, const v
 tsa_status run_scatter(const tsa_params* p, const void* oc, const int32_t* idx, const int32_t* k_seq, void* o,
                        uint32_t* status, cudaStream_t st) {
   tsa::ScatterArgs a{static_cast<const __nv_bfloat16*>(oc), idx, kept_of(p, k_seq),
-                     static_cast<__nv_bfloat16*>(o), status, p->L, p->Hq};
+                     static_cast<__nv_bfloat16*>(o), strides_of(token_major(p), p->Hq, p->L, p->d), status,
+                     p->L, p->Hq};
   const dim3 g((p->L + tsa::SCAT_ROWS - 1) / tsa::SCAT_ROWS, p->B * p->Hq);
   if (p->d == 128)
     tsa::scatter_kernel<128><<<g, 256, 0, st>>>(a);
@@ -279,9 +299,12 @@ tsa_status run_scatter(const tsa_params* p, const void* oc, const int32_t* idx, 
 // idx (with scatter): output row i lands at row idx[i] of o (the rest of o is
 // not touched).  idx with gather as well: Q/K/V rows are loaded by index from
 // the uncompressed tensors instead of as compressed tiles.
+// in_tm / out_tm: q, k, v / o are token-major (the caller's layout) rather
+// than head-major (compressed buffers).
 tsa_status run_attend(const tsa_params* p, const void* q, const void* k, const void* v, int heads_kv, int g_kv,
                       const int32_t* k_seq, void* o, float* lse, uint32_t* status, uint32_t* abort_word,
-                      cudaStream_t st, const int32_t* idx = nullptr, bool gather = false) {
+                      cudaStream_t st, bool in_tm, bool out_tm, const int32_t* idx = nullptr,
+                      bool gather = false) {
   CUtensorMap mq, mk, mv;
   const int bhq = p->B * p->Hq;
   const int bhkv = p->B * heads_kv;
@@ -291,8 +314,9 @@ tsa_status run_attend(const tsa_params* p, const void* q, const void* k, const v
       gather ? (make_row_map(&mq, q, p->d, static_cast<long long>(bhq) * p->L) &&
                 make_row_map(&mk, k, p->d, static_cast<long long>(bhkv) * p->L) &&
                 make_row_map(&mv, v, p->d, static_cast<long long>(bhkv) * p->L))
-             : (make_map(&mq, q, p->d, p->L, bhq) && make_map(&mk, k, p->d, p->L, bhkv) &&
-                make_map(&mv, v, p->d, p->L, bhkv));
+             : (make_map(&mq, q, p->d, p->L, p->Hq, p->B, in_tm) &&
+                make_map(&mk, k, p->d, p->L, heads_kv, p->B, in_tm) &&
+                make_map(&mv, v, p->d, p->L, heads_kv, p->B, in_tm));
   if (!maps_ok) return TSA_ERR_CUDA;
   if (cudaMemsetAsync(abort_word, 0, sizeof(uint32_t), st) != cudaSuccess) return TSA_ERR_CUDA;
   tsa::AttnArgs a;
@@ -310,6 +334,8 @@ tsa_status run_attend(const tsa_params* p, const void* q, const void* k, const v
   a.scale_log2 = scale_of(p) * 1.4426950408889634f;
   a.limit_ns = limit_ns_of(p);
   a.test_stall = (p->flags & TSA_FLAG_TEST_STALL) ? 1 : 0;
+  a.token_major = in_tm ? 1 : 0;
+  a.os = strides_of(out_tm, p->Hq, p->L, p->d);
   const dim3 grid((a.n_tiles + 1) / 2, bhq);  // two query tiles per CTA
   auto launch = [&](auto kernel, std::atomic<int>(&attr)[kMaxDevices], int threads, int smem) -> tsa_status {
     if (!ensure_smem(attr, kernel, smem)) return TSA_ERR_CUDA;
@@ -332,7 +358,8 @@ tsa_status run_attend(const tsa_params* p, const void* q, const void* k, const v
 // they are).
 tsa_status run_zero_unselected(const tsa_params* p, const int32_t* idx, const int32_t* k_seq, void* o,
                                uint32_t* status, cudaStream_t st) {
-  tsa::ScatterArgs a{nullptr, idx, kept_of(p, k_seq), static_cast<__nv_bfloat16*>(o), status, p->L, p->Hq};
+  tsa::ScatterArgs a{nullptr, idx, kept_of(p, k_seq), static_cast<__nv_bfloat16*>(o),
+                     strides_of(token_major(p), p->Hq, p->L, p->d), status, p->L, p->Hq};
   const dim3 g((p->L + tsa::SCAT_ROWS - 1) / tsa::SCAT_ROWS, p->B * p->Hq);
   if (p->d == 128)
     tsa::scatter_kernel<128, true><<<g, 256, 0, st>>>(a);
@@ -388,6 +415,7 @@ tsa_status tsa_check_params(const tsa_params* p) {
   if ((p->flags & ~TSA_FLAG_TEST_STALL) != 0) return TSA_ERR_INVALID_ARG;
   if (p->budget_mode < TSA_BUDGET_MAX || p->budget_mode > TSA_BUDGET_PER_HEAD) return TSA_ERR_INVALID_ARG;
   if (p->keep_recent < 0 || p->keep_recent > p->L) return TSA_ERR_INVALID_ARG;
+  if (p->layout != TSA_LAYOUT_BHLD && p->layout != TSA_LAYOUT_BLHD) return TSA_ERR_INVALID_ARG;
   if (p->d != 64 && p->d != 128) return TSA_ERR_UNSUPPORTED;
   if (p->w > 4096 || p->L > (1 << 22)) return TSA_ERR_UNSUPPORTED;
   if (static_cast<long long>(p->B) * p->Hq * p->L >= (1LL << 31)) return TSA_ERR_UNSUPPORTED;
@@ -474,7 +502,7 @@ tsa_status tsa_attend(const tsa_params* p, const void* qc, const void* kc, const
   if (!tensors_ok({qc, kc, vc, k_seq, oc}) || (lse && !aligned(lse, 4))) return TSA_ERR_INVALID_ARG;
   if ((s = check_ws(p, ws, ws_bytes, false)) != TSA_OK) return s;
   return run_attend(p, qc, kc, vc, p->Hq, 1, k_seq, oc, lse, status_of(ws), abort_of(ws),
-                    static_cast<cudaStream_t>(stream));
+                    static_cast<cudaStream_t>(stream), false, false);
 }
 
 tsa_status tsa_attend_dense(const tsa_params* p, const void* q, const void* k, const void* v, void* o,
@@ -484,7 +512,7 @@ tsa_status tsa_attend_dense(const tsa_params* p, const void* q, const void* k, c
   if (!tensors_ok({q, k, v, o}) || (lse && !aligned(lse, 4))) return TSA_ERR_INVALID_ARG;
   if ((s = check_ws(p, ws, ws_bytes, false)) != TSA_OK) return s;
   return run_attend(p, q, k, v, p->Hkv, p->Hq / p->Hkv, nullptr, o, lse, status_of(ws), abort_of(ws),
-                    static_cast<cudaStream_t>(stream));
+                    static_cast<cudaStream_t>(stream), token_major(p), token_major(p));
 }
 
 tsa_status tsa_scatter(const tsa_params* p, const void* oc, const int32_t* idx, const int32_t* k_seq, void* o,
@@ -523,7 +551,8 @@ tsa_status tsa_forward(const tsa_params* p, const void* q, const void* k, const 
   void* kc = at<void>(ws, w.kc);
   void* vc = at<void>(ws, w.vc);
   if ((s = run_gather(p, q, k, v, idx, kseq, qc, kc, vc, status_of(ws), st)) != TSA_OK) return s;
-  if ((s = run_attend(p, qc, kc, vc, p->Hq, 1, kseq, o, nullptr, status_of(ws), abort_of(ws), st, idx)) != TSA_OK)
+  if ((s = run_attend(p, qc, kc, vc, p->Hq, 1, kseq, o, nullptr, status_of(ws), abort_of(ws), st, false,
+                      token_major(p), idx)) != TSA_OK)
     return s;
   return run_zero_unselected(p, idx, kseq, o, status_of(ws), st);
 }
@@ -536,7 +565,8 @@ tsa_status tsa_attend_scatter(const tsa_params* p, const void* qc, const void* k
   if (!tensors_ok({qc, kc, vc, idx, k_seq, o}) || (lse && !aligned(lse, 4))) return TSA_ERR_INVALID_ARG;
   if ((s = check_ws(p, ws, ws_bytes, false)) != TSA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if ((s = run_attend(p, qc, kc, vc, p->Hq, 1, k_seq, o, lse, status_of(ws), abort_of(ws), st, idx)) != TSA_OK)
+  if ((s = run_attend(p, qc, kc, vc, p->Hq, 1, k_seq, o, lse, status_of(ws), abort_of(ws), st, false,
+                      token_major(p), idx)) != TSA_OK)
     return s;
   return run_zero_unselected(p, idx, k_seq, o, status_of(ws), st);
 }
@@ -549,8 +579,8 @@ tsa_status tsa_attend_gathered(const tsa_params* p, const void* q, const void* k
   if (!tensors_ok({q, k, v, idx, k_seq, o}) || (lse && !aligned(lse, 4))) return TSA_ERR_INVALID_ARG;
   if ((s = check_ws(p, ws, ws_bytes, false)) != TSA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if ((s = run_attend(p, q, k, v, p->Hkv, p->Hq / p->Hkv, k_seq, o, lse, status_of(ws), abort_of(ws), st, idx,
-                      true)) != TSA_OK)
+  if ((s = run_attend(p, q, k, v, p->Hkv, p->Hq / p->Hkv, k_seq, o, lse, status_of(ws), abort_of(ws), st,
+                      token_major(p), token_major(p), idx, true)) != TSA_OK)
     return s;
   return run_zero_unselected(p, idx, k_seq, o, status_of(ws), st);
 }
