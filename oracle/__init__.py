@@ -17,7 +17,8 @@ budget, per-head selection).  The abstract pages with the same title
 compress / attend / decompress scheme in summary form.
 
 Readings taken where the page is silent (each is also pinned by a test):
-  * "recent queries" = the last w query positions; the proxy map is causal
+  * "recent queries" = the last w query positions (all of them when the
+    sequence is shorter than w); the proxy map is causal
     (window row at position i sees keys j <= i) and uses the attention's
     own scale 1/sqrt(d) (fp32 value, widened).
   * importance of key j = sum over the w window rows of the row-normalised
@@ -105,7 +106,7 @@ def proxy_scores(q, k, w: int, scale: float | None = None, return_f64: bool = Fa
     out64 = np.empty((B, Hq, L), dtype=np.float64) if return_f64 else None
     for b in range(B):
         for h in range(Hq):
-            r = proxy_scores_head(q[b, h, L - w:], k[b, h // G], L, scale, return_f64)
+            r = proxy_scores_head(q[b, h, max(L - w, 0):], k[b, h // G], L, scale, return_f64)
             if return_f64:
                 out[b, h], out64[b, h] = r
             else:
@@ -307,6 +308,35 @@ def forward(q, k, v, w: int, tau: float, scale: float | None = None, mode: str =
     oc = compressed_attention(qc, kc, vc, kept, scale)
     o = scatter(oc, idx, kept, L)
     return dict(scores=scores, k_head=k_head, k_seq=k_seq, kept=kept, idx=idx, oc=oc, o=o)
+
+
+def forward_varlen(q, k, v, cu_seqlens, w: int, tau: float, scale: float | None = None, mode: str = "max",
+                   keep_recent: int = 0) -> list:
+    """A batch of sequences of different lengths, packed token-major: q
+    [T, Hq, d], k and v [T, Hkv, d], sequence b at tokens
+    [cu_seqlens[b], cu_seqlens[b+1]).  Every sequence is independent, so each
+    runs the whole path on its own; returns one ``forward`` result per
+    sequence (arrays in the head-major layout of that sequence) and the
+    packed output [T, Hq, d] under the key "o_packed" of the first."""
+    cu = [int(c) for c in cu_seqlens]
+    T, Hq, d = q.shape
+    o_packed = np.zeros((T, Hq, d), dtype=np.float64)
+    res = []
+    for b in range(len(cu) - 1):
+        t0, t1 = cu[b], cu[b + 1]
+        hm = lambda x: np.ascontiguousarray(x[t0:t1].transpose(1, 0, 2))[None]   # [1, H, L_b, d]
+        if t1 == t0:                              # an empty sequence keeps nothing
+            z = np.zeros((1, Hq), dtype=np.int32)
+            r = dict(scores=np.zeros((1, Hq, 0), np.float32), k_head=z, k_seq=np.zeros(1, np.int32), kept=z,
+                     idx=np.zeros((1, Hq, 0), np.int32), oc=np.zeros((1, Hq, 0, d)), o=np.zeros((1, Hq, 0, d)))
+            res.append(r)
+            continue
+        r = forward(hm(q), hm(k), hm(v), w, tau, scale, mode, min(keep_recent, t1 - t0))
+        o_packed[t0:t1] = r["o"][0].transpose(1, 0, 2)
+        res.append(r)
+    if res:
+        res[0]["o_packed"] = o_packed
+    return res
 
 
 def output_rows(q, k, v, idx, k_seq, b: int, h: int, orig_rows, scale: float | None = None):

@@ -196,3 +196,69 @@ def test_planted_mistakes_are_caught():
     def shared_always(k_head, k_seq, mode="max"):
         return O.kept_counts(k_head, k_seq, "max")
     assert _fails(check_mode_fixtures, O.coverage_budget, shared_always, O.select_topk)
+
+
+def test_window_longer_than_sequence_covers_it():
+    """A sequence shorter than the window: every query row is a window row,
+    so each of the L rows of the proxy map sums to one and the scores sum
+    to L; pinned against a pure-Python brute force of the definition."""
+    import math
+    rng = np.random.default_rng(11)
+    from workloads import f32_to_bf16_bits, bf16_bits_to_f64
+    L, d = 5, 8
+    q = f32_to_bf16_bits(rng.standard_normal((1, 1, L, d)).astype(np.float32))
+    k = f32_to_bf16_bits(rng.standard_normal((1, 1, L, d)).astype(np.float32))
+    s32, s64 = O.proxy_scores(q, k, 9, return_f64=True)
+    assert abs(s64[0, 0].sum() - L) < 1e-12
+    qf, kf, sc = bf16_bits_to_f64(q)[0, 0], bf16_bits_to_f64(k)[0, 0], O.default_scale(d)
+    brute = [0.0] * L
+    for i in range(L):
+        xs = [sum(qf[i, t] * kf[j, t] for t in range(d)) * sc for j in range(i + 1)]
+        m = max(xs)
+        z = sum(math.exp(x - m) for x in xs)
+        for j in range(i + 1):
+            brute[j] += math.exp(xs[j] - m) / z
+    assert np.allclose(s64[0, 0], brute, rtol=1e-12, atol=1e-14)
+
+
+def test_varlen_equal_lengths_matches_batched_forward():
+    """Packed sequences of equal length give exactly the batched result."""
+    rng = np.random.default_rng(12)
+    from workloads import f32_to_bf16_bits
+    B, Hq, Hkv, L, d = 3, 4, 2, 40, 64
+    mk = lambda *s: f32_to_bf16_bits(rng.standard_normal(s).astype(np.float32))
+    q, k, v = mk(B, Hq, L, d), mk(B, Hkv, L, d), mk(B, Hkv, L, d)
+    ref = O.forward(q, k, v, 8, 0.2, mode="per_head", keep_recent=3)
+    pk = lambda x: np.ascontiguousarray(x.transpose(0, 2, 1, 3).reshape(B * L, x.shape[1], d))
+    res = O.forward_varlen(pk(q), pk(k), pk(v), [0, L, 2 * L, 3 * L], 8, 0.2, mode="per_head", keep_recent=3)
+    for b in range(B):
+        assert np.array_equal(res[b]["idx"][0], ref["idx"][b])
+        assert np.array_equal(res[b]["kept"][0], ref["kept"][b])
+        assert np.array_equal(res[b]["o"][0], ref["o"][b])
+    assert np.array_equal(res[0]["o_packed"], ref["o"].transpose(0, 2, 1, 3).reshape(B * L, Hq, d))
+
+
+def test_varlen_sequences_are_independent():
+    """Changing one sequence's tokens leaves every other sequence's result
+    unchanged, and the packed output is zero outside the selections."""
+    rng = np.random.default_rng(13)
+    from workloads import f32_to_bf16_bits
+    Hq, Hkv, d = 2, 1, 64
+    cu = [0, 17, 17, 60, 61]
+    T = cu[-1]
+    mk = lambda *s: f32_to_bf16_bits(rng.standard_normal(s).astype(np.float32))
+    q, k, v = mk(T, Hq, d), mk(T, Hkv, d), mk(T, Hkv, d)
+    a = O.forward_varlen(q, k, v, cu, 8, 0.1)
+    q2 = q.copy()
+    q2[17:60] = mk(43, Hq, d)
+    b = O.forward_varlen(q2, k, v, cu, 8, 0.1)
+    for s in (0, 1, 3):
+        assert np.array_equal(a[s]["o"], b[s]["o"])
+    assert a[1]["o"].shape[2] == 0                      # an empty sequence
+    o = a[0]["o_packed"]
+    for s in range(len(cu) - 1):
+        n = int(a[s]["k_seq"][0])
+        for h in range(Hq):
+            sel = cu[s] + a[s]["idx"][0, h, :n]
+            rest = np.setdiff1d(np.arange(cu[s], cu[s + 1]), sel)
+            assert (o[rest, h] == 0).all()
