@@ -26,6 +26,16 @@
  *            [B, L, Hq, d] and k, v [B, L, Hkv, d], the layout a prefill
  *            engine's projections produce.  Only the caller's q, k, v, o
  *            follow p->layout; every tensor below is always head-major.
+ *            Varlen batches (p->cu_seqlens not NULL, token-major only):
+ *            sequences of different lengths packed one after another, q, o
+ *            [T, Hq, d] and k, v [T, Hkv, d] with T = p->total_tokens;
+ *            sequence b is tokens [cu_seqlens[b], cu_seqlens[b+1]) and its
+ *            length L_b is at most p->L, which then is the capacity of every
+ *            per-head buffer below (entries past L_b are not meaningful).  A
+ *            sequence shorter than w uses all its tokens as the window.
+ *            Every call reads cu_seqlens on the device; a sequence that does
+ *            not fit in [0, T] or is longer than L is treated as empty and
+ *            sets TSA_DEVFLAG_BAD_INDEX (in tsa_budget).
  *   scores   fp32 [B, Hq, L]
  *   idx      int32 [B, Hq, L]: entries [0, k_b) hold S_h ascending, the rest -1
  *   k_head   int32 [B, Hq]            k_seq  int32 [B]
@@ -120,6 +130,9 @@ typedef struct tsa_params {
                            are kept in every head (each k_head is raised to
                            at least r; the selection ranks them first)       */
   int32_t layout;       /* TSA_LAYOUT_BHLD (0) or TSA_LAYOUT_BLHD (1)        */
+  int32_t total_tokens; /* varlen: T, the packed tensors' token count; else 0 */
+  const int32_t* cu_seqlens; /* varlen: DEVICE int32 [B+1] token offsets,
+                           non-decreasing from 0; NULL for B sequences of L  */
 } tsa_params;
 
 /* Version of this ABI (TSA_ABI_VERSION of the built library). */

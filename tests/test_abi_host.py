@@ -64,6 +64,9 @@ def test_status_strings(lib):
     (dict(budget_mode="per_head"), 0), (dict(keep_recent=-1), INVALID), (dict(keep_recent=4097), INVALID),
     (dict(keep_recent=4096), 0), (dict(keep_recent=64, budget_mode="per_head"), 0),
     (dict(layout="blhd"), 0), (dict(layout=2), INVALID), (dict(layout=-1), INVALID),
+    (dict(cu_seqlens=FAKE, total_tokens=9000), 0), (dict(cu_seqlens=FAKE, total_tokens=0), INVALID),
+    (dict(cu_seqlens=FAKE + 2, total_tokens=10), INVALID), (dict(total_tokens=5), INVALID),
+    (dict(cu_seqlens=FAKE, total_tokens=1 << 30), UNSUPPORTED),
 ])
 def test_param_validation(lib, kw, want):
     p = good(**kw)

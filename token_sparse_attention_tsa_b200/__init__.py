@@ -47,18 +47,32 @@ class tsa_params(ctypes.Structure):
                 ("L", ctypes.c_int32), ("d", ctypes.c_int32), ("w", ctypes.c_int32),
                 ("tau", ctypes.c_float), ("softmax_scale", ctypes.c_float),
                 ("flags", ctypes.c_uint32), ("timeout_ms", ctypes.c_uint32),
-                ("budget_mode", ctypes.c_int32), ("keep_recent", ctypes.c_int32), ("layout", ctypes.c_int32)]
+                ("budget_mode", ctypes.c_int32), ("keep_recent", ctypes.c_int32), ("layout", ctypes.c_int32),
+                ("total_tokens", ctypes.c_int32), ("cu_seqlens", ctypes.c_void_p)]
 
 
 def params(B, Hq, Hkv, L, d, w, tau, softmax_scale=0.0, timeout_ms=0, flags=0, budget_mode=BUDGET_MAX,
-           keep_recent=0, layout=LAYOUT_BHLD) -> tsa_params:
+           keep_recent=0, layout=LAYOUT_BHLD, cu_seqlens=None, total_tokens=0) -> tsa_params:
     """budget_mode: BUDGET_MAX / BUDGET_MEAN / BUDGET_PER_HEAD or "max" / "mean" / "per_head".
-    layout: LAYOUT_BHLD / LAYOUT_BLHD or "bhld" / "blhd" (memory order of q, k, v, o)."""
+    layout: LAYOUT_BHLD / LAYOUT_BLHD or "bhld" / "blhd" (memory order of q, k, v, o).
+    cu_seqlens: for a packed varlen batch, a CUDA int32 tensor [B+1] (kept
+    alive by the caller while the params are used), with total_tokens = T
+    and L = the longest sequence; the layout is then token-major."""
     if isinstance(budget_mode, str):
         budget_mode = BUDGET_MODES[budget_mode]
     if isinstance(layout, str):
         layout = LAYOUTS[layout]
-    return tsa_params(B, Hq, Hkv, L, d, w, tau, softmax_scale, flags, timeout_ms, budget_mode, keep_recent, layout)
+    cu = None
+    if cu_seqlens is not None:
+        cu = cu_seqlens if isinstance(cu_seqlens, int) else _ptr(cu_seqlens, "cu_seqlens", _torch().int32)
+        layout = LAYOUT_BLHD
+    return tsa_params(B, Hq, Hkv, L, d, w, tau, softmax_scale, flags, timeout_ms, budget_mode, keep_recent, layout,
+                      total_tokens, cu)
+
+
+def _torch():
+    import torch
+    return torch
 
 
 _lock = threading.Lock()
@@ -310,3 +324,30 @@ def forward(q, k, v, w: int, tau: float, softmax_scale: float = 0.0, ws=None, re
     k_seq = torch.empty(kshape, dtype=torch.int32, device=q.device)
     tsa_forward(p, q, k, v, o, ws, scores, idx, k_seq)
     return o, scores, idx, k_seq
+
+
+def forward_varlen(q, k, v, cu_seqlens, max_seqlen: int, w: int, tau: float, softmax_scale: float = 0.0,
+                   ws=None, return_intermediates=False, budget_mode=BUDGET_MAX, keep_recent: int = 0):
+    """Convenience wrapper for a packed varlen batch: q [T, Hq, d], k and v
+    [T, Hkv, d], cu_seqlens a CUDA int32 tensor [B+1] of token offsets and
+    max_seqlen the longest sequence.  Returns o [T, Hq, d] (and, with
+    intermediates, scores, idx, kept as in ``forward`` with capacity
+    max_seqlen)."""
+    import torch
+    T_tok, Hq, d = q.shape
+    Hkv = k.shape[1]
+    B = cu_seqlens.numel() - 1
+    p = params(B, Hq, Hkv, max_seqlen, d, w, tau, softmax_scale, budget_mode=budget_mode,
+               keep_recent=keep_recent, cu_seqlens=cu_seqlens, total_tokens=T_tok)
+    if ws is None:
+        ws = new_workspace(p, full=True, device=q.device)
+    o = torch.empty_like(q)
+    if not return_intermediates:
+        tsa_forward(p, q, k, v, o, ws)
+        return o
+    scores = torch.empty((B, Hq, max_seqlen), dtype=torch.float32, device=q.device)
+    idx = torch.empty((B, Hq, max_seqlen), dtype=torch.int32, device=q.device)
+    kshape = (B, Hq) if p.budget_mode == BUDGET_PER_HEAD else (B,)
+    kept = torch.empty(kshape, dtype=torch.int32, device=q.device)
+    tsa_forward(p, q, k, v, o, ws, scores, idx, kept)
+    return o, scores, idx, kept

@@ -40,6 +40,8 @@ struct AttnArgs {
   uint64_t limit_ns;      // per-wait time limit
   int test_stall;         // failure-path test: the MMA issuer first waits on a barrier nothing completes
   int token_major;        // Q/K/V maps are (d, H, L, B) (else (d, L, H, B)); gather rows likewise
+  int in_packed;          // Q/K/V are packed sequences (token coordinate cu[b] + t, one map "sequence")
+  Seqs seqs;              // sequence lengths L_b (and packed token offsets)
 };
 
 // ---------------------------------------------------------------------------
@@ -122,7 +124,8 @@ __global__ void __launch_bounds__(Attn2Layout<D>::THREADS, 1)
   const int n_pairs = (a.n_tiles + 1) >> 1;
   const int t0 = 2 * (n_pairs - 1 - static_cast<int>(blockIdx.x));  // longest pairs first
 
-  const int valid = a.kept.of(b, h, a.L);
+  const int seq_len = a.seqs.len(b);
+  const int valid = a.kept.of(b, h, seq_len);
   if (t0 * C::BM >= valid) return;                 // uniform, before any barrier
   const bool two = (t0 + 1) * C::BM < valid;       // second query tile has rows
   const int last0 = t0;                            // tile 0 attends KV tiles 0..t0
@@ -182,7 +185,8 @@ __global__ void __launch_bounds__(Attn2Layout<D>::THREADS, 1)
           if (leader) {
 #pragma unroll
             for (int c = 0; c < C::NCH; ++c)
-              tma_load_rows(dst + c * C::CHUNK, m, br, tm, c * 64, tile * C::BM, hz, b);
+              tma_load_rows(dst + c * C::CHUNK, m, br, tm, c * 64, a.in_packed ? a.seqs.map_t(b, tile * C::BM) : tile * C::BM,
+                            hz, a.in_packed ? 0 : b);
           }
         } else {
           int rr[4];
@@ -190,8 +194,9 @@ __global__ void __launch_bounds__(Attn2Layout<D>::THREADS, 1)
           for (int u = 0; u < 4; ++u) {
             const int i = tile * C::BM + 4 * lane + u;
             int v = i < valid ? __ldg(a.idx + static_cast<size_t>(bh) * a.L + i) : 0;
-            v = (v >= 0 && v < a.L) ? v : 0;
-            rr[u] = tm ? (b * a.L + v) * nh + hz : (b * nh + hz) * a.L + v;
+            v = (v >= 0 && v < seq_len) ? v : 0;
+            const int tok = a.in_packed ? a.seqs.tok0(b) + v : b * a.L + v;
+            rr[u] = tm ? tok * nh + hz : (b * nh + hz) * a.L + v;
           }
 #pragma unroll 4
           for (int g = 0; g < 32; ++g) {
@@ -439,7 +444,7 @@ __global__ void __launch_bounds__(Attn2Layout<D>::THREADS, 1)
       bool store = row < valid;
       if constexpr (kScatter) {  // compressed row i goes to token S_h[i]
         orow_index = store ? __ldg(a.idx + static_cast<size_t>(bh) * a.L + row) : 0;
-        if (store && (orow_index < 0 || orow_index >= a.L)) {
+        if (store && (orow_index < 0 || orow_index >= seq_len)) {
           store = false;
           if (a.status) atomicOr(a.status, 0x4u);
         }

@@ -24,6 +24,7 @@ struct GatherArgs {
   RowStrides qs, kvs;              // their row strides (head-major or token-major)
   const int32_t* idx;              // [B*Hq, L]
   Kept kept;                       // rows kept per (b, h)
+  Seqs seqs;                       // sequence lengths L_b
   __nv_bfloat16 *qc, *kc, *vc;     // [B*Hq, L, D]; qc may be null (K and V only)
   uint32_t* status;                // or null
   int L, Hq, Hkv, G;
@@ -42,10 +43,11 @@ __global__ void __launch_bounds__(256) gather_kernel(const GatherArgs a) {
     const int i = static_cast<int>(row - bh * a.L);
     const int b = static_cast<int>(bh / a.Hq);
     const int h = static_cast<int>(bh - static_cast<long long>(b) * a.Hq);
-    if (i >= a.kept.of(b, h, a.L)) continue;
+    const int Lb = a.seqs.len(b);
+    if (i >= a.kept.of(b, h, Lb)) continue;
     const int j = __ldg(a.idx + row);
     const size_t dst = static_cast<size_t>(row) * D + sub * 8;
-    if (j < 0 || j >= a.L) {
+    if (j < 0 || j >= Lb) {
       bad = true;
       const uint4 z = make_uint4(0, 0, 0, 0);
       if (a.qc) *reinterpret_cast<uint4*>(a.qc + dst) = z;
@@ -72,6 +74,7 @@ struct ScatterArgs {
   RowStrides os;            // row strides of o (head-major or token-major)
   uint32_t* status;         // or null
   int L, Hq;
+  Seqs seqs;                // sequence lengths L_b: rows [0, L_b) of o are written
 };
 
 constexpr int SCAT_ROWS = 256;  // output rows per CTA
@@ -89,7 +92,8 @@ __global__ void __launch_bounds__(256) scatter_kernel(const ScatterArgs a) {
   const int bh = blockIdx.y;
   const int r0 = blockIdx.x * SCAT_ROWS;
   const int b = bh / a.Hq;
-  const int kb = a.kept.of(b, bh - b * a.Hq, a.L);
+  const int Lb = a.seqs.len(b);
+  const int kb = a.kept.of(b, bh - b * a.Hq, Lb);
   const int32_t* ix = a.idx + static_cast<size_t>(bh) * a.L;
   where[threadIdx.x] = -1;
   if (threadIdx.x == 0) {  // first i with ix[i] >= r0
@@ -107,7 +111,7 @@ __global__ void __launch_bounds__(256) scatter_kernel(const ScatterArgs a) {
     if (i < kb) {
       const int r = __ldg(ix + i) - r0;
       if (r >= 0 && r < SCAT_ROWS) where[r] = i;
-      else if (r + r0 < 0 || r + r0 >= a.L) bad = true;
+      else if (r + r0 < 0 || r + r0 >= Lb) bad = true;
     }
   }
   __syncthreads();
@@ -115,7 +119,7 @@ __global__ void __launch_bounds__(256) scatter_kernel(const ScatterArgs a) {
   constexpr int ROWS_PER_PASS = 256 / LPR;
   for (int rr = threadIdx.x / LPR; rr < SCAT_ROWS; rr += ROWS_PER_PASS) {
     const int r = r0 + rr;
-    if (r >= a.L) break;
+    if (r >= Lb) break;
     const int i = where[rr];
     if (kZeroOnly && i >= 0) continue;
     uint4 val = make_uint4(0, 0, 0, 0);

@@ -6,9 +6,9 @@
 // recent queries against all keys; a key's importance is the sum of its
 // column of attention weights.
 //
-// Here: for each (b, h) and window row i in [L-w, L), x_ij = scale *
+// Here: for each (b, h) and window row i in [L_b-w_b, L_b), x_ij = scale *
 // q[b,h,i].k[b,h/G,j] over keys j <= i; p_ij = softmax_j(x_ij);
-// score[b,h,j] = sum_i p_ij.
+// score[b,h,j] = sum_i p_ij (L_b the sequence's length, w_b = min(w, L_b)).
 //
 // The logits come from tcgen05 tensor cores (bf16 products are exact; fp32
 // accumulation).  To keep the scores within 1e-5 relative of the exact value,
@@ -49,6 +49,7 @@ struct ScoreArgs {
   float scale_log2;        // scale * log2(e)
   uint64_t limit_ns;
   int token_major;         // q, k maps are (d, H, L, B) (else (d, L, H, B))
+  Seqs seqs;               // sequence lengths (and packed token offsets)
 };
 
 template <int D>
@@ -105,8 +106,11 @@ __global__ void __launch_bounds__(SC_THREADS, 1)
   const int chunk = blockIdx.x;
   const int bh = blockIdx.y;
   const int b = bh / a.Hq, h = bh - (bh / a.Hq) * a.Hq;
+  const int Lb = a.seqs.len(b);                  // this sequence's length
+  const int wb = a.w < Lb ? a.w : Lb;              // its window
+  const int pos0 = Lb - wb;                        // position of window row 0
   const int key0 = chunk * SC_CHUNK_TILES * SC_KEYS;
-  int n_kt = (a.L - key0 + SC_KEYS - 1) / SC_KEYS;
+  int n_kt = Lb > key0 ? (Lb - key0 + SC_KEYS - 1) / SC_KEYS : 0;
   n_kt = n_kt > SC_CHUNK_TILES ? SC_CHUNK_TILES : n_kt;
   const int steps = n_kt * a.n_rb;
   auto step_rb = [&](int s) { return kPass2 ? s % a.n_rb : s / n_kt; };
@@ -151,13 +155,14 @@ __global__ void __launch_bounds__(SC_THREADS, 1)
       if (leader) {
         const uint32_t sb = base + st * C::STAGE;
         mbar_arrive_expect_tx(bar(SB_FULL + st), C::STAGE);
-        const int qrow = a.L - a.w + step_rb(s) * SC_ROWS;   // may be < 0 only if w > L (rejected)
-        const int krow = key0 + step_kt(s) * SC_KEYS;
+        const int qrow = a.seqs.map_t(b, pos0 + step_rb(s) * SC_ROWS);
+        const int krow = a.seqs.map_t(b, key0 + step_kt(s) * SC_KEYS);
+        const int bc = a.seqs.map_b(b);
 #pragma unroll
         for (int c = 0; c < C::NCH; ++c) {
-          tma_load_rows(sb + c * C::CHUNK, &tmQ, bar(SB_FULL + st), a.token_major, c * 64, qrow, h, b);
+          tma_load_rows(sb + c * C::CHUNK, &tmQ, bar(SB_FULL + st), a.token_major, c * 64, qrow, h, bc);
           tma_load_rows(sb + C::Q_BYTES + c * C::K_CHUNK, &tmK, bar(SB_FULL + st), a.token_major, c * 64, krow,
-                        h / a.G, b);
+                        h / a.G, bc);
         }
       }
       issued = s + 1;
@@ -210,8 +215,8 @@ __global__ void __launch_bounds__(SC_THREADS, 1)
     for (int s = 0; s < steps; ++s) {
       const int buf = s & 1, rb = step_rb(s), kt = step_kt(s);
       const int wr = rb * SC_ROWS + r;              // window row
-      const int pos = a.L - a.w + wr;               // its position
-      const bool row_ok = wr < a.w;
+      const int pos = pos0 + wr;                    // its position
+      const bool row_ok = wr < wb;
       // the four row warps agree before going on, so the shared-memory column
       // exchange below can never leave a warp waiting alone
       const bool ok = __all_sync(0xffffffffu, mbar_wait(bar(SB_S + buf), (s >> 1) & 1, wc));
@@ -250,7 +255,7 @@ __global__ void __launch_bounds__(SC_THREADS, 1)
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const int key = kbase + c * 32 + e;
-            x[c][e] = (row_ok && key <= pos && key < a.L) ? x[c][e] * sl2 : -INFINITY;
+            x[c][e] = (row_ok && key <= pos && key < Lb) ? x[c][e] * sl2 : -INFINITY;
             mx = fmaxf(mx, x[c][e]);
           }
         if (mx != -INFINITY) {
@@ -277,8 +282,8 @@ __global__ void __launch_bounds__(SC_THREADS, 1)
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
             const int key = kbase + c * 32 + e;
-            x[c][e] = (row_ok && key <= pos && key < a.L) ? ex2_approx(fmaf(x[c][e], sl2, -st_row.x)) * st_row.y
-                                                         : 0.f;
+            x[c][e] = (row_ok && key <= pos && key < Lb) ? ex2_approx(fmaf(x[c][e], sl2, -st_row.x)) * st_row.y
+                                                        : 0.f;
           }
           colsum[c] += warp_column_sums(x[c], lane);
         }
@@ -292,7 +297,7 @@ __global__ void __launch_bounds__(SC_THREADS, 1)
           if (warp < 2) {
             const int col = warp * 32 + lane;
             const float v = (red[col] + red[SC_KEYS + col]) + (red[2 * SC_KEYS + col] + red[3 * SC_KEYS + col]);
-            if (kbase + col < a.L) a.scores[static_cast<size_t>(bh) * a.L + kbase + col] = v;
+            if (kbase + col < Lb) a.scores[static_cast<size_t>(bh) * a.L + kbase + col] = v;
           }
           colsum[0] = colsum[1] = 0.f;
         }
@@ -314,16 +319,20 @@ __global__ void __launch_bounds__(SC_THREADS, 1)
   }
 }
 
-// Merge the chunk statistics: one thread per (head, window row).
+// Merge the chunk statistics: one thread per (head, window row), over the
+// key chunks its sequence has.
 static __global__ void score_merge_kernel(const ScoreArgs a, int total_rows) {
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= total_rows) return;
+  const int Lb = a.seqs.len(idx / a.w / a.Hq);
+  constexpr int span = SC_CHUNK_TILES * SC_KEYS;
+  const int nc = (Lb + span - 1) / span;
   const float* pm = a.part_m + static_cast<size_t>(idx) * a.n_chunks;
   const double* pz = a.part_z + static_cast<size_t>(idx) * a.n_chunks;
   float m = -INFINITY;
-  for (int c = 0; c < a.n_chunks; ++c) m = fmaxf(m, pm[c]);
+  for (int c = 0; c < nc; ++c) m = fmaxf(m, pm[c]);
   double z = 0.0;
-  for (int c = 0; c < a.n_chunks; ++c)
+  for (int c = 0; c < nc; ++c)
     if (pm[c] != -INFINITY) z += pz[c] * exp2(static_cast<double>(pm[c]) - m);
   a.stats[idx] = make_float2(m, static_cast<float>(1.0 / z));
 }

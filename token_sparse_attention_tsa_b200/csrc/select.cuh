@@ -99,12 +99,13 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* r
 }
 
 struct BudgetArgs {
-  const float* scores;  // [B*Hq, L]
+  const float* scores;  // [B*Hq, L]: the first L_b entries of each row are read
   int32_t* k_head;      // [B*Hq]
   uint32_t* status;     // or null
   int L, Hq;
-  int keep_recent;      // r in [0, L]: every k_head is raised to at least r
+  int keep_recent;      // r in [0, L]: every k_head is raised to at least min(r, L_b)
   double tau;           // fp32 tau widened
+  Seqs seqs;            // sequence lengths L_b
 };
 
 // grid: B*Hq CTAs of 1024 threads; dynamic smem: per-warp histograms.
@@ -119,10 +120,11 @@ __global__ void __launch_bounds__(BS_THREADS, 1) budget_kernel(const BudgetArgs 
   const int bh = blockIdx.x;
   const float* sc = a.scores + static_cast<size_t>(bh) * a.L;
   const int warp = threadIdx.x >> 5;
-  bool bad = false;
+  bool bad = false, bad_seq = false;
+  const int Lb = a.seqs.len_ok(bh / a.Hq, bad_seq);
 
   unsigned long long tot = 0;
-  for (int j = threadIdx.x; j < a.L; j += BS_THREADS) tot += mass_of_key(score_key(sc[j], bad));
+  for (int j = threadIdx.x; j < Lb; j += BS_THREADS) tot += mass_of_key(score_key(sc[j], bad));
   tot = block_sum<unsigned long long>(tot, red64);
   const unsigned long long T =
       static_cast<unsigned long long>(floor(__dmul_rn(a.tau, __ull2double_rn(tot))));
@@ -143,7 +145,7 @@ __global__ void __launch_bounds__(BS_THREADS, 1) budget_kernel(const BudgetArgs 
     }
     __syncthreads();
     const uint32_t prefix = s_prefix, mask = s_mask;
-    for (int j = threadIdx.x; j < a.L; j += BS_THREADS) {
+    for (int j = threadIdx.x; j < Lb; j += BS_THREADS) {
       const uint32_t u = score_key(sc[j], bad);
       if ((u & mask) == prefix) {
         const uint32_t dgt = (u >> shift) & 255u;
@@ -194,8 +196,10 @@ __global__ void __launch_bounds__(BS_THREADS, 1) budget_kernel(const BudgetArgs 
       const unsigned long long qstar = mass_of_key(s_prefix);  // > 0 here
       p += static_cast<uint32_t>(s_rem / qstar);
     }
-    const int32_t kh = a.L - static_cast<int32_t>(p);
-    a.k_head[bh] = kh > a.keep_recent ? kh : a.keep_recent;
+    const int32_t kh = Lb - static_cast<int32_t>(p);
+    const int32_t r = a.keep_recent < Lb ? a.keep_recent : Lb;
+    a.k_head[bh] = kh > r ? kh : r;
+    if (bad_seq && a.status) atomicOr(a.status, 0x4u);
   }
   if (a.status && __syncthreads_or(bad) && threadIdx.x == 0) atomicOr(a.status, 0x1u);
 }
@@ -222,11 +226,12 @@ __global__ void __launch_bounds__(32) budget_finalize_kernel(const int32_t* k_he
 }
 
 struct SelectArgs {
-  const float* scores;   // [B*Hq, L]
+  const float* scores;   // [B*Hq, L]: the first L_b entries of each row are read
   Kept kept;             // rows kept per (b, h)
   int32_t* idx;          // [B*Hq, L]
   int L, Hq;
-  int keep_recent;       // tokens [L - r, L) rank above every score
+  int keep_recent;       // tokens [L_b - r, L_b) rank above every score
+  Seqs seqs;             // sequence lengths L_b
 };
 
 // Selection key: the score's order key, or the top key for a forced token
@@ -244,20 +249,21 @@ __global__ void __launch_bounds__(BS_THREADS, 1) select_kernel(const SelectArgs 
   __shared__ uint32_t s_rem, s_prefix, s_mask;
 
   const int bh = blockIdx.x;
-  const int L = a.L;
-  const float* sc = a.scores + static_cast<size_t>(bh) * L;
-  int32_t* out = a.idx + static_cast<size_t>(bh) * L;
+  const int cap = a.L;                               // row capacity of idx
+  const int L = a.seqs.len(bh / a.Hq);               // this sequence's length
+  const float* sc = a.scores + static_cast<size_t>(bh) * cap;
+  int32_t* out = a.idx + static_cast<size_t>(bh) * cap;
   const int k = a.kept.of(bh / a.Hq, bh % a.Hq, L);
-  const int first_forced = L - a.keep_recent;
+  const int first_forced = L - (a.keep_recent < L ? a.keep_recent : L);
   const int warp = threadIdx.x >> 5;
   bool bad = false;
 
   if (k == L) {  // everything kept
-    for (int i = threadIdx.x; i < L; i += BS_THREADS) out[i] = i;
+    for (int i = threadIdx.x; i < cap; i += BS_THREADS) out[i] = i < L ? i : -1;
     return;
   }
   if (k == 0) {
-    for (int i = threadIdx.x; i < L; i += BS_THREADS) out[i] = -1;
+    for (int i = threadIdx.x; i < cap; i += BS_THREADS) out[i] = -1;
     return;
   }
   if (threadIdx.x == 0) {
@@ -329,7 +335,7 @@ __global__ void __launch_bounds__(BS_THREADS, 1) select_kernel(const SelectArgs 
     }
     if (take) out[pos++] = j;
   }
-  for (int i = k + threadIdx.x; i < L; i += BS_THREADS) out[i] = -1;
+  for (int i = k + threadIdx.x; i < cap; i += BS_THREADS) out[i] = -1;
 }
 
 }  // namespace tsa

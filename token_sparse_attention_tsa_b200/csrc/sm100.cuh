@@ -370,26 +370,55 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
   return d;
 }
 
+// Sequences of a batch: B sequences of L tokens each, or (cu not null)
+// packed sequences, sequence b at tokens [cu[b], cu[b+1]) of T in all, each
+// at most L long.  A packed sequence that does not fit in [0, T] or is longer
+// than L counts as empty (len_ok reports it).
+struct Seqs {
+  const int32_t* cu;
+  int L, T;
+  __device__ __forceinline__ int len_ok(int b, bool& bad) const {
+    if (!cu) return L;
+    const int t0 = __ldg(cu + b), t1 = __ldg(cu + b + 1);
+    const bool ok = t0 >= 0 && t1 >= t0 && t1 <= T && t1 - t0 <= L;
+    bad |= !ok;
+    return ok ? t1 - t0 : 0;
+  }
+  __device__ __forceinline__ int len(int b) const {
+    bool bad = false;
+    return len_ok(b, bad);
+  }
+  __device__ __forceinline__ int tok0(int b) const { return cu ? __ldg(cu + b) : 0; }
+  // coordinates of token t of sequence b in a 4D tensor map: packed maps
+  // have one "sequence" spanning all T tokens
+  __device__ __forceinline__ int map_t(int b, int t) const { return cu ? __ldg(cu + b) + t : t; }
+  __device__ __forceinline__ int map_b(int b) const { return cu ? 0 : b; }
+};
+
 // Element offset of row (sequence b, head h, token t) of a bf16 tensor with
 // element strides sb, sh, st (head-major [B, H, L, d]: H*L*d, L*d, d;
-// token-major [B, L, H, d]: L*H*d, d, H*d).
+// token-major [B, L, H, d]: L*H*d, d, H*d).  With cu (packed token-major
+// sequences [T, H, d]) token t of sequence b is packed token cu[b] + t.
 struct RowStrides {
   long long sb, sh, st;
+  const int32_t* cu;
   __device__ __forceinline__ size_t at(int b, int h, int t) const {
+    if (cu) return static_cast<size_t>((__ldg(cu + b) + static_cast<long long>(t)) * st + h * sh);
     return static_cast<size_t>(b * sb + h * sh + t * st);
   }
 };
 
 // Rows kept by each (sequence b, head h): n[b * sb + h * sh], clipped to
-// [0, L].  Per-sequence counts use (sb, sh) = (1, 0), per-head counts
-// (Hq, 1); a null n keeps every row (the dense case).
+// [0, len] (len: the sequence's length).  Per-sequence counts use
+// (sb, sh) = (1, 0), per-head counts (Hq, 1); a null n keeps every row (the
+// dense case).
 struct Kept {
   const int32_t* n;
   int sb, sh;
-  __device__ __forceinline__ int of(int b, int h, int L) const {
-    if (!n) return L;
+  __device__ __forceinline__ int of(int b, int h, int len) const {
+    if (!n) return len;
     const int k = __ldg(n + static_cast<size_t>(b) * sb + static_cast<size_t>(h) * sh);
-    return k < 0 ? 0 : (k > L ? L : k);
+    return k < 0 ? 0 : (k > len ? len : k);
   }
 };
 

@@ -83,7 +83,20 @@ bool token_major(const tsa_params* p) { return p->layout == TSA_LAYOUT_BLHD; }
 
 tsa::RowStrides strides_of(bool tm, int heads, int L, int d) {
   const long long H = heads, Ll = L, dd = d;
-  return tm ? tsa::RowStrides{Ll * H * dd, dd, H * dd} : tsa::RowStrides{H * Ll * dd, Ll * dd, dd};
+  return tm ? tsa::RowStrides{Ll * H * dd, dd, H * dd, nullptr} : tsa::RowStrides{H * Ll * dd, Ll * dd, dd, nullptr};
+}
+
+// Packed varlen batch: the caller's q, k, v, o hold total_tokens tokens,
+// sequence b at [cu_seqlens[b], cu_seqlens[b+1]).
+bool packed(const tsa_params* p) { return p->cu_seqlens != nullptr; }
+
+tsa::Seqs seqs_of(const tsa_params* p) { return tsa::Seqs{p->cu_seqlens, p->L, p->total_tokens}; }
+
+// Row strides of the caller's tensors (with `heads` heads).
+tsa::RowStrides caller_strides(const tsa_params* p, int heads) {
+  tsa::RowStrides r = strides_of(token_major(p), heads, p->L, p->d);
+  r.cu = p->cu_seqlens;
+  return r;
 }
 
 // Kept-row counts as the kernels read them: per sequence [B], or per head
@@ -174,14 +187,21 @@ constexpr int kBudgetSmem = tsa::BS_WARPS * 256 * (8 + 4);
 constexpr int kSelectSmem = tsa::BS_WARPS * 256 * 4;
 
 // ---------------------------------------------------------------- launchers
+// Tensor map over the caller's q, k or v (`heads` heads): per-sequence
+// batches in either layout, or packed sequences as one token-major sequence
+// of total_tokens tokens.
+bool make_caller_map(CUtensorMap* m, const tsa_params* p, const void* base, int heads, int box_rows = 128) {
+  if (packed(p)) return make_map(m, base, p->d, p->total_tokens, heads, 1, true, box_rows);
+  return make_map(m, base, p->d, p->L, heads, p->B, token_major(p), box_rows);
+}
+
 tsa_status run_score(const tsa_params* p, const void* q, const void* k, float* scores, void* ws,
                      cudaStream_t st) {
   const WsLayout w = layout_of(p);
   const int bhq = p->B * p->Hq;
   CUtensorMap mq, mk;
   const bool tm = token_major(p);
-  if (!make_map(&mq, q, p->d, p->L, p->Hq, p->B, tm, tsa::SC_ROWS) ||
-      !make_map(&mk, k, p->d, p->L, p->Hkv, p->B, tm, tsa::SC_KEYS))
+  if (!make_caller_map(&mq, p, q, p->Hq, tsa::SC_ROWS) || !make_caller_map(&mk, p, k, p->Hkv, tsa::SC_KEYS))
     return TSA_ERR_CUDA;
   tsa::ScoreArgs a;
   a.scores = scores;
@@ -200,6 +220,7 @@ tsa_status run_score(const tsa_params* p, const void* q, const void* k, float* s
   a.scale_log2 = scale_of(p) * 1.4426950408889634f;
   a.limit_ns = limit_ns_of(p);
   a.token_major = tm ? 1 : 0;
+  a.seqs = seqs_of(p);
   const dim3 grid(a.n_chunks, bhq);
   const int rows = bhq * p->w;
   if (cudaMemsetAsync(a.abort_word, 0, sizeof(uint32_t), st) != cudaSuccess) return TSA_ERR_CUDA;
@@ -229,7 +250,7 @@ tsa_status run_score(const tsa_params* p, const void* q, const void* k, float* s
 tsa_status run_budget(const tsa_params* p, const float* scores, int32_t* k_head, int32_t* k_seq,
                       uint32_t* status, cudaStream_t st) {
   if (!ensure_smem(g_budget, tsa::budget_kernel, kBudgetSmem)) return TSA_ERR_CUDA;
-  tsa::BudgetArgs a{scores, k_head, status, p->L, p->Hq, p->keep_recent, static_cast<double>(p->tau)};
+  tsa::BudgetArgs a{scores, k_head, status, p->L, p->Hq, p->keep_recent, static_cast<double>(p->tau), seqs_of(p)};
   tsa::budget_kernel<<<p->B * p->Hq, tsa::BS_THREADS, kBudgetSmem, st>>>(a);
   if (k_seq)
     tsa::budget_finalize_kernel<<<p->B, 32, 0, st>>>(k_head, k_seq, p->Hq,
@@ -240,7 +261,7 @@ tsa_status run_budget(const tsa_params* p, const float* scores, int32_t* k_head,
 tsa_status run_select(const tsa_params* p, const float* scores, const int32_t* kept, int32_t* idx,
                       cudaStream_t st) {
   if (!ensure_smem(g_select, tsa::select_kernel, kSelectSmem)) return TSA_ERR_CUDA;
-  tsa::SelectArgs a{scores, kept_of(p, kept), idx, p->L, p->Hq, p->keep_recent};
+  tsa::SelectArgs a{scores, kept_of(p, kept), idx, p->L, p->Hq, p->keep_recent, seqs_of(p)};
   tsa::select_kernel<<<p->B * p->Hq, tsa::BS_THREADS, kSelectSmem, st>>>(a);
   return launch_ok();
 }
@@ -259,8 +280,9 @@ tsa_status run_gather(const tsa_params* p, const void* q, const void* k, const v
   a.v = static_cast<const __nv_bfloat16*>(v);
   a.idx = idx;
   a.kept = kept_of(p, k_seq);
-  a.qs = strides_of(token_major(p), p->Hq, p->L, p->d);
-  a.kvs = strides_of(token_major(p), p->Hkv, p->L, p->d);
+  a.seqs = seqs_of(p);
+  a.qs = caller_strides(p, p->Hq);
+  a.kvs = caller_strides(p, p->Hkv);
   a.qc = static_cast<__nv_bfloat16*>(qc);
   a.kc = static_cast<__nv_bfloat16*>(kc);
   a.vc = static_cast<__nv_bfloat16*>(vc);
@@ -280,8 +302,7 @@ tsa_status run_gather(const tsa_params* p, const void* q, const void* k, const v
 tsa_status run_scatter(const tsa_params* p, const void* oc, const int32_t* idx, const int32_t* k_seq, void* o,
                        uint32_t* status, cudaStream_t st) {
   tsa::ScatterArgs a{static_cast<const __nv_bfloat16*>(oc), idx, kept_of(p, k_seq),
-                     static_cast<__nv_bfloat16*>(o), strides_of(token_major(p), p->Hq, p->L, p->d), status,
-                     p->L, p->Hq};
+                     static_cast<__nv_bfloat16*>(o), caller_strides(p, p->Hq), status, p->L, p->Hq, seqs_of(p)};
   const dim3 g((p->L + tsa::SCAT_ROWS - 1) / tsa::SCAT_ROWS, p->B * p->Hq);
   if (p->d == 128)
     tsa::scatter_kernel<128><<<g, 256, 0, st>>>(a);
@@ -299,24 +320,24 @@ tsa_status run_scatter(const tsa_params* p, const void* oc, const int32_t* idx, 
 // idx (with scatter): output row i lands at row idx[i] of o (the rest of o is
 // not touched).  idx with gather as well: Q/K/V rows are loaded by index from
 // the uncompressed tensors instead of as compressed tiles.
-// in_tm / out_tm: q, k, v / o are token-major (the caller's layout) rather
-// than head-major (compressed buffers).
+// in_caller / out_caller: q, k, v / o are the caller's tensors (p->layout,
+// possibly packed sequences) rather than head-major compressed buffers.
 tsa_status run_attend(const tsa_params* p, const void* q, const void* k, const void* v, int heads_kv, int g_kv,
                       const int32_t* k_seq, void* o, float* lse, uint32_t* status, uint32_t* abort_word,
-                      cudaStream_t st, bool in_tm, bool out_tm, const int32_t* idx = nullptr,
+                      cudaStream_t st, bool in_caller, bool out_caller, const int32_t* idx = nullptr,
                       bool gather = false) {
   CUtensorMap mq, mk, mv;
-  const int bhq = p->B * p->Hq;
-  const int bhkv = p->B * heads_kv;
   const bool scatter = idx != nullptr;
   gather = gather && scatter;
+  const long long tokens = (in_caller && packed(p)) ? p->total_tokens : static_cast<long long>(p->B) * p->L;
   const bool maps_ok =
-      gather ? (make_row_map(&mq, q, p->d, static_cast<long long>(bhq) * p->L) &&
-                make_row_map(&mk, k, p->d, static_cast<long long>(bhkv) * p->L) &&
-                make_row_map(&mv, v, p->d, static_cast<long long>(bhkv) * p->L))
-             : (make_map(&mq, q, p->d, p->L, p->Hq, p->B, in_tm) &&
-                make_map(&mk, k, p->d, p->L, heads_kv, p->B, in_tm) &&
-                make_map(&mv, v, p->d, p->L, heads_kv, p->B, in_tm));
+      gather ? (make_row_map(&mq, q, p->d, tokens * p->Hq) && make_row_map(&mk, k, p->d, tokens * heads_kv) &&
+                make_row_map(&mv, v, p->d, tokens * heads_kv))
+      : in_caller ? (make_caller_map(&mq, p, q, p->Hq) && make_caller_map(&mk, p, k, heads_kv) &&
+                     make_caller_map(&mv, p, v, heads_kv))
+                  : (make_map(&mq, q, p->d, p->L, p->Hq, p->B, false) &&
+                     make_map(&mk, k, p->d, p->L, heads_kv, p->B, false) &&
+                     make_map(&mv, v, p->d, p->L, heads_kv, p->B, false));
   if (!maps_ok) return TSA_ERR_CUDA;
   if (cudaMemsetAsync(abort_word, 0, sizeof(uint32_t), st) != cudaSuccess) return TSA_ERR_CUDA;
   tsa::AttnArgs a;
@@ -334,9 +355,11 @@ tsa_status run_attend(const tsa_params* p, const void* q, const void* k, const v
   a.scale_log2 = scale_of(p) * 1.4426950408889634f;
   a.limit_ns = limit_ns_of(p);
   a.test_stall = (p->flags & TSA_FLAG_TEST_STALL) ? 1 : 0;
-  a.token_major = in_tm ? 1 : 0;
-  a.os = strides_of(out_tm, p->Hq, p->L, p->d);
-  const dim3 grid((a.n_tiles + 1) / 2, bhq);  // two query tiles per CTA
+  a.token_major = (in_caller && token_major(p)) ? 1 : 0;
+  a.in_packed = (in_caller && packed(p)) ? 1 : 0;
+  a.seqs = seqs_of(p);
+  a.os = out_caller ? caller_strides(p, p->Hq) : strides_of(false, p->Hq, p->L, p->d);
+  const dim3 grid((a.n_tiles + 1) / 2, p->B * p->Hq);  // two query tiles per CTA
   auto launch = [&](auto kernel, std::atomic<int>(&attr)[kMaxDevices], int threads, int smem) -> tsa_status {
     if (!ensure_smem(attr, kernel, smem)) return TSA_ERR_CUDA;
     kernel<<<grid, threads, smem, st>>>(mq, mk, mv, a);
@@ -358,8 +381,8 @@ tsa_status run_attend(const tsa_params* p, const void* q, const void* k, const v
 // they are).
 tsa_status run_zero_unselected(const tsa_params* p, const int32_t* idx, const int32_t* k_seq, void* o,
                                uint32_t* status, cudaStream_t st) {
-  tsa::ScatterArgs a{nullptr, idx, kept_of(p, k_seq), static_cast<__nv_bfloat16*>(o),
-                     strides_of(token_major(p), p->Hq, p->L, p->d), status, p->L, p->Hq};
+  tsa::ScatterArgs a{nullptr, idx, kept_of(p, k_seq), static_cast<__nv_bfloat16*>(o), caller_strides(p, p->Hq),
+                     status, p->L, p->Hq, seqs_of(p)};
   const dim3 g((p->L + tsa::SCAT_ROWS - 1) / tsa::SCAT_ROWS, p->B * p->Hq);
   if (p->d == 128)
     tsa::scatter_kernel<128, true><<<g, 256, 0, st>>>(a);
@@ -416,6 +439,14 @@ tsa_status tsa_check_params(const tsa_params* p) {
   if (p->budget_mode < TSA_BUDGET_MAX || p->budget_mode > TSA_BUDGET_PER_HEAD) return TSA_ERR_INVALID_ARG;
   if (p->keep_recent < 0 || p->keep_recent > p->L) return TSA_ERR_INVALID_ARG;
   if (p->layout != TSA_LAYOUT_BHLD && p->layout != TSA_LAYOUT_BLHD) return TSA_ERR_INVALID_ARG;
+  if (p->cu_seqlens) {  // packed sequences: token-major, at least one token, offsets 4-byte aligned
+    if (p->layout != TSA_LAYOUT_BLHD || p->total_tokens < 1 || !aligned(p->cu_seqlens, 4))
+      return TSA_ERR_INVALID_ARG;
+    if (static_cast<long long>(p->total_tokens) * (p->Hq > p->Hkv ? p->Hq : p->Hkv) >= (1LL << 31))
+      return TSA_ERR_UNSUPPORTED;
+  } else if (p->total_tokens != 0) {
+    return TSA_ERR_INVALID_ARG;
+  }
   if (p->d != 64 && p->d != 128) return TSA_ERR_UNSUPPORTED;
   if (p->w > 4096 || p->L > (1 << 22)) return TSA_ERR_UNSUPPORTED;
   if (static_cast<long long>(p->B) * p->Hq * p->L >= (1LL << 31)) return TSA_ERR_UNSUPPORTED;
@@ -512,7 +543,7 @@ tsa_status tsa_attend_dense(const tsa_params* p, const void* q, const void* k, c
   if (!tensors_ok({q, k, v, o}) || (lse && !aligned(lse, 4))) return TSA_ERR_INVALID_ARG;
   if ((s = check_ws(p, ws, ws_bytes, false)) != TSA_OK) return s;
   return run_attend(p, q, k, v, p->Hkv, p->Hq / p->Hkv, nullptr, o, lse, status_of(ws), abort_of(ws),
-                    static_cast<cudaStream_t>(stream), token_major(p), token_major(p));
+                    static_cast<cudaStream_t>(stream), true, true);
 }
 
 tsa_status tsa_scatter(const tsa_params* p, const void* oc, const int32_t* idx, const int32_t* k_seq, void* o,
@@ -551,8 +582,8 @@ tsa_status tsa_forward(const tsa_params* p, const void* q, const void* k, const 
   void* kc = at<void>(ws, w.kc);
   void* vc = at<void>(ws, w.vc);
   if ((s = run_gather(p, q, k, v, idx, kseq, qc, kc, vc, status_of(ws), st)) != TSA_OK) return s;
-  if ((s = run_attend(p, qc, kc, vc, p->Hq, 1, kseq, o, nullptr, status_of(ws), abort_of(ws), st, false,
-                      token_major(p), idx)) != TSA_OK)
+  if ((s = run_attend(p, qc, kc, vc, p->Hq, 1, kseq, o, nullptr, status_of(ws), abort_of(ws), st, false, true,
+                      idx)) != TSA_OK)
     return s;
   return run_zero_unselected(p, idx, kseq, o, status_of(ws), st);
 }
@@ -565,8 +596,8 @@ tsa_status tsa_attend_scatter(const tsa_params* p, const void* qc, const void* k
   if (!tensors_ok({qc, kc, vc, idx, k_seq, o}) || (lse && !aligned(lse, 4))) return TSA_ERR_INVALID_ARG;
   if ((s = check_ws(p, ws, ws_bytes, false)) != TSA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if ((s = run_attend(p, qc, kc, vc, p->Hq, 1, k_seq, o, lse, status_of(ws), abort_of(ws), st, false,
-                      token_major(p), idx)) != TSA_OK)
+  if ((s = run_attend(p, qc, kc, vc, p->Hq, 1, k_seq, o, lse, status_of(ws), abort_of(ws), st, false, true,
+                      idx)) != TSA_OK)
     return s;
   return run_zero_unselected(p, idx, k_seq, o, status_of(ws), st);
 }
@@ -579,8 +610,8 @@ tsa_status tsa_attend_gathered(const tsa_params* p, const void* q, const void* k
   if (!tensors_ok({q, k, v, idx, k_seq, o}) || (lse && !aligned(lse, 4))) return TSA_ERR_INVALID_ARG;
   if ((s = check_ws(p, ws, ws_bytes, false)) != TSA_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if ((s = run_attend(p, q, k, v, p->Hkv, p->Hq / p->Hkv, k_seq, o, lse, status_of(ws), abort_of(ws), st,
-                      token_major(p), token_major(p), idx, true)) != TSA_OK)
+  if ((s = run_attend(p, q, k, v, p->Hkv, p->Hq / p->Hkv, k_seq, o, lse, status_of(ws), abort_of(ws), st, true,
+                      true, idx, true)) != TSA_OK)
     return s;
   return run_zero_unselected(p, idx, k_seq, o, status_of(ws), st);
 }
