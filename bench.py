@@ -205,6 +205,73 @@ def run_reference(args, wl, rank: int) -> int:
     return 0
 
 
+# ---------------------------------------------------------------- varlen leg
+def run_varlen(args, wl) -> int:
+    """One packed varlen batch (sequence b: the first L_b tokens of sequence b
+    of the workload), timed like the headline step on one GPU.  Effective
+    TFLOP/s counts the dense causal FLOPs of every sequence."""
+    import torch
+    import token_sparse_attention_tsa_b200 as T
+    lengths = [int(x) for x in args.varlen.split(",")]
+    Lmax = max(lengths)
+    wl = wl.with_(B=len(lengths), L=Lmax)
+    qh, kh, vh = W.generate(wl)
+    pack = lambda x: np.ascontiguousarray(np.concatenate(
+        [x[b, :, :n].transpose(1, 0, 2) for b, n in enumerate(lengths)], axis=0))
+    q, k, v = (torch.from_numpy(pack(x)).view(torch.bfloat16).cuda() for x in (qh, kh, vh))
+    del qh, kh, vh
+    cu = torch.tensor(np.concatenate([[0], np.cumsum(lengths)]), dtype=torch.int32, device="cuda")
+    p = T.params(wl.B, wl.Hq, wl.Hkv, Lmax, wl.d, wl.w, args.tau, budget_mode=args.budget_mode,
+                 keep_recent=args.keep_recent, cu_seqlens=cu, total_tokens=q.shape[0])
+    ws = T.new_workspace(p, full=True)
+    o = torch.empty_like(q)
+    scores = torch.empty((wl.B, wl.Hq, Lmax), device="cuda")
+    idx = torch.empty((wl.B, wl.Hq, Lmax), dtype=torch.int32, device="cuda")
+    kept = torch.empty((wl.B, wl.Hq) if args.budget_mode == "per_head" else (wl.B,), dtype=torch.int32,
+                       device="cuda")
+    fwd = lambda: T.tsa_forward(p, q, k, v, o, ws, scores, idx, kept)
+    for _ in range(args.warmup):
+        fwd()
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    with ClockSampler(0) as clk:
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(args.steps):
+            fwd()
+        b.record(stream)
+        torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / args.steps
+    status, flags = T.get_device_status(ws)
+    if status != 0:
+        print(json.dumps({"error": f"device status {status} flags {flags}"}), file=sys.stderr)
+        return 3
+    kept_np = kept.cpu().numpy()
+    per_head = kept_np if kept_np.ndim == 2 else np.repeat(kept_np[:, None], wl.Hq, axis=1)
+    dense = sum(wl.Hq * 2.0 * wl.d * n * (n + 1) for n in lengths)
+    comp = float((2.0 * wl.d * per_head.astype(np.float64) * (per_head + 1)).sum())
+    od = torch.empty_like(q)
+    for _ in range(2):
+        T.tsa_attend_dense(p, q, k, v, od, None, ws)
+    torch.cuda.synchronize()
+    a.record(stream)
+    T.tsa_attend_dense(p, q, k, v, od, None, ws)
+    b.record(stream)
+    torch.cuda.synchronize()
+    dense_ms = a.elapsed_time(b)
+    line = {"metric": METRIC + " (packed varlen batch)", "value": dense / (ms * 1e-3) / 1e12, "unit": UNIT,
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "varlen_lengths": lengths, "Hq": wl.Hq, "Hkv": wl.Hkv, "d": wl.d,
+                       "w": wl.w, "tau": args.tau, "budget_mode": args.budget_mode, "layout": "packed token-major"},
+            "kept_rows_fraction": float(per_head.sum()) / (wl.Hq * sum(lengths)),
+            "achieved_tflops": comp / (ms * 1e-3) / 1e12, "dense_ms": dense_ms,
+            "speedup_vs_dense": dense_ms / ms, "gpu_launches": KERNELS_PER_FORWARD * args.steps,
+            "clocks": clk.summary()}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 # ---------------------------------------------------------------- GPU leg
 def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
     import torch
@@ -231,11 +298,13 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
     # inputs: this rank's own sequence
     wl_r = rank_workload(wl, rank)
     qh, kh, vh = W.generate(wl_r)
+    if args.layout == "blhd":   # the caller's tensors token-major [B, L, H, d]
+        qh, kh, vh = (np.ascontiguousarray(x.transpose(0, 2, 1, 3)) for x in (qh, kh, vh))
     pin = [torch.from_numpy(x).view(torch.bfloat16).pin_memory() for x in (qh, kh, vh)]
     q, k, v = [x.to(dev, non_blocking=True) for x in pin]
     o = torch.empty_like(q)
     p = T.params(wl.B, wl.Hq, wl.Hkv, wl.L, wl.d, wl.w, args.tau, budget_mode=args.budget_mode,
-                 keep_recent=args.keep_recent)
+                 keep_recent=args.keep_recent, layout=args.layout)
     ws = T.new_workspace(p, full=True, device=dev)
     scores = torch.empty((wl.B, wl.Hq, wl.L), dtype=torch.float32, device=dev)
     idx = torch.empty((wl.B, wl.Hq, wl.L), dtype=torch.int32, device=dev)
@@ -328,14 +397,16 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
     try:  # library baseline (context only); fused backends only, never the O(L^2)-memory one
         from torch.nn.attention import SDPBackend, sdpa_kernel
         sdpa = torch.nn.functional.scaled_dot_product_attention
+        hm = (lambda x: x.transpose(1, 2)) if args.layout == "blhd" else (lambda x: x)
+        sq, sk, sv = hm(q), hm(k), hm(v)
         with sdpa_kernel([SDPBackend.CUDNN_ATTENTION, SDPBackend.FLASH_ATTENTION]):
-            sdpa(q, k, v, is_causal=True, enable_gqa=True)
-            sdpa_ms = timed(lambda: sdpa(q, k, v, is_causal=True, enable_gqa=True), 2)
+            sdpa(sq, sk, sv, is_causal=True, enable_gqa=True)
+            sdpa_ms = timed(lambda: sdpa(sq, sk, sv, is_causal=True, enable_gqa=True), 2)
     except Exception:
         sdpa_ms = None
 
     # ---- end to end: pinned host inputs -> device -> tsa_forward -> host output
-    o_host = torch.empty(shape, dtype=torch.bfloat16).pin_memory()
+    o_host = torch.empty(tuple(o.shape), dtype=torch.bfloat16).pin_memory()
 
     def e2e_step():
         q.copy_(pin[0], non_blocking=True)
@@ -389,6 +460,7 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "L": wl.L, "d": wl.d, "w": wl.w,
                    "tau": args.tau, "budget_mode": args.budget_mode, "keep_recent": args.keep_recent,
+                   "layout": args.layout,
                    "parallelism": f"replicas{world}" if world > 1 else "single",
                    "l2": "inputs larger than L2 (Q 1 GiB, K/V 256 MiB each)"},
         "k_seq": ks, "keep_fraction": [x / wl.L for x in ks],
@@ -422,6 +494,10 @@ def main() -> int:
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--budget-mode", default="max", choices=["max", "mean", "per_head"])
     ap.add_argument("--keep-recent", type=int, default=0)
+    ap.add_argument("--layout", default="bhld", choices=["bhld", "blhd"])
+    ap.add_argument("--varlen", default=None,
+                    help="comma-separated sequence lengths: time a packed varlen batch of the workload's "
+                         "first L_b tokens per sequence instead of the headline step")
     args = ap.parse_args()
     wl = W.WORKLOADS[args.workload]
     if args.tau is None:
@@ -432,6 +508,8 @@ def main() -> int:
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         return run_reference(args, wl, rank)
+    if args.varlen:
+        return run_varlen(args, wl)
     return run_gpu(args, wl, rank, world, local_rank)
 
 
