@@ -43,6 +43,9 @@ Readings taken where the page is silent (each is also pinned by a test):
   * GQA: selection per Q head h; K and V rows come from KV head h // G.
   * scatter: a zero L x d output per head; row S_h[i] receives row i of
     the compressed output; every other row is exactly zero.
+  * block-sparse composition (optional): a block mask over 128-token blocks
+    of compressed positions; compressed row i attends key j <= i only when
+    j's block is i's own block or the mask allows the pair of blocks.
 
 Every function here is pinned in ``tests/test_oracle_pins.py`` against brute
 force, closed forms, hand-derived fixtures (``tests/golden``) and an
@@ -226,11 +229,16 @@ def gather_qkv(q, k, v, idx, k_seq):
 # Step 5: causal attention over the compressed set.  [GS] "Arquitectura
 # Central": the compressed tensors are attended by an ordinary dense kernel.
 # ---------------------------------------------------------------------------
+BLOCK = 128   # block edge of the block-sparse composition
+
+
 def attention_rows(qc: np.ndarray, kc: np.ndarray, vc: np.ndarray, rows, scale: float,
-                   chunk: int = 1024) -> np.ndarray:
+                   chunk: int = 1024, block_mask: np.ndarray | None = None) -> np.ndarray:
     """Causal softmax attention for the listed rows of one head (fp64).
 
-    Row i: o_i = sum_{j<=i} softmax_j(scale * q_i . k_j) v_j.
+    Row i: o_i = sum_{j<=i, allowed} softmax_j(scale * q_i . k_j) v_j, where
+    with a block mask [NB, NB] key j is allowed when j // 128 == i // 128 or
+    block_mask[i // 128, j // 128] is nonzero (every key otherwise).
     Rows are evaluated independently; ``chunk`` only bounds memory.
     """
     rows = np.asarray(rows, dtype=np.int64)
@@ -242,15 +250,20 @@ def attention_rows(qc: np.ndarray, kc: np.ndarray, vc: np.ndarray, rows, scale: 
         kf = _f64(kc[:n])
         vf = _f64(vc[:n])
         x = (qf @ kf.T) * scale
-        x = np.where(np.arange(n)[None, :] <= r[:, None], x, -np.inf)
+        allow = np.arange(n)[None, :] <= r[:, None]
+        if block_mask is not None:
+            qb, kb = r[:, None] // BLOCK, np.arange(n)[None, :] // BLOCK
+            allow &= (qb == kb) | (np.asarray(block_mask)[qb, kb] != 0)
+        x = np.where(allow, x, -np.inf)
         m = x.max(axis=1, keepdims=True)
         e = np.exp(x - m)
         out[c0:c0 + chunk] = (e @ vf) / e.sum(axis=1, keepdims=True)
     return out
 
 
-def compressed_attention(qc, kc, vc, k_seq, scale: float | None = None) -> np.ndarray:
-    """O_hat [B,Hq,L,d] fp64; rows >= k_b are zero."""
+def compressed_attention(qc, kc, vc, k_seq, scale: float | None = None, block_mask=None) -> np.ndarray:
+    """O_hat [B,Hq,L,d] fp64; rows >= k_b are zero.  block_mask: optional
+    [B, Hq, NB, NB] over 128-token blocks of compressed positions."""
     B, Hq, L, d = qc.shape
     if scale is None:
         scale = default_scale(d)
@@ -258,8 +271,9 @@ def compressed_attention(qc, kc, vc, k_seq, scale: float | None = None) -> np.nd
     for b in range(B):
         for h in range(Hq):
             kb = _kept(k_seq, b, h)
+            bm = None if block_mask is None else block_mask[b, h]
             oc[b, h, :kb] = attention_rows(qc[b, h, :kb], kc[b, h, :kb], vc[b, h, :kb],
-                                           np.arange(kb), scale)
+                                           np.arange(kb), scale, block_mask=bm)
     return oc
 
 

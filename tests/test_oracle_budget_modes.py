@@ -262,3 +262,73 @@ def test_varlen_sequences_are_independent():
             sel = cu[s] + a[s]["idx"][0, h, :n]
             rest = np.setdiff1d(np.arange(cu[s], cu[s + 1]), sel)
             assert (o[rest, h] == 0).all()
+
+
+# --------------------------------------------------------------------------
+# block-sparse composition over the compressed sequence
+# --------------------------------------------------------------------------
+def _rand_bf16(rng, *shape):
+    from workloads import f32_to_bf16_bits
+    return f32_to_bf16_bits(rng.standard_normal(shape).astype(np.float32))
+
+
+def test_block_mask_all_ones_is_plain_attention():
+    rng = np.random.default_rng(21)
+    B, H, L, d = 1, 2, 300, 64
+    q, k, v = (_rand_bf16(rng, B, H, L, d) for _ in range(3))
+    nb = (L + 127) // 128
+    kept = np.array([L, 260]).reshape(1, 2)
+    ref = O.compressed_attention(q, k, v, kept)
+    got = O.compressed_attention(q, k, v, kept, block_mask=np.ones((B, H, nb, nb), np.uint8))
+    assert np.array_equal(ref, got)
+
+
+def test_block_diagonal_mask_is_local_attention_torch():
+    """Only the diagonal blocks: every 128-row block attends causally within
+    itself, checked block by block against torch fp64 SDPA."""
+    rng = np.random.default_rng(22)
+    from workloads import bf16_bits_to_f64
+    L, d = 333, 64
+    q, k, v = (_rand_bf16(rng, 1, 1, L, d) for _ in range(3))
+    nb = (L + 127) // 128
+    got = O.compressed_attention(q, k, v, np.array([L]), block_mask=np.zeros((1, 1, nb, nb), np.uint8))
+    for s in range(0, L, 128):
+        e = min(L, s + 128)
+        t = lambda x: torch.from_numpy(bf16_bits_to_f64(x[0, 0, s:e]))[None, None]
+        ref = torch.nn.functional.scaled_dot_product_attention(t(q), t(k), t(v), is_causal=True,
+                                                               scale=O.default_scale(d))[0, 0].numpy()
+        assert np.abs(got[0, 0, s:e] - ref).max() < 1e-12
+
+
+def test_block_mask_brute_force():
+    """A random mask against a pure-Python loop over the definition."""
+    import math
+    rng = np.random.default_rng(23)
+    from workloads import bf16_bits_to_f64
+    L, d = 290, 8
+    q, k, v = (_rand_bf16(rng, 1, 1, L, d) for _ in range(3))
+    nb = (L + 127) // 128
+    bm = (rng.random((1, 1, nb, nb)) < 0.5).astype(np.uint8)
+    got = O.compressed_attention(q, k, v, np.array([L]), block_mask=bm)
+    qf, kf, vf = (bf16_bits_to_f64(x)[0, 0] for x in (q, k, v))
+    sc = O.default_scale(d)
+    for i in (0, 127, 128, 200, 255, 256, 289):
+        keys = [j for j in range(i + 1) if j // 128 == i // 128 or bm[0, 0, i // 128, j // 128]]
+        xs = [sum(qf[i, t] * kf[j, t] for t in range(d)) * sc for j in keys]
+        m = max(xs)
+        ws = [math.exp(x - m) for x in xs]
+        z = sum(ws)
+        ref = [sum(ws[a] * vf[j, t] for a, j in enumerate(keys)) / z for t in range(d)]
+        assert np.allclose(got[0, 0, i], ref, rtol=1e-12, atol=1e-13)
+
+
+def test_block_mask_planted_mistake_is_caught():
+    """A mask read transposed (key block, query block) fails the brute force."""
+    rng = np.random.default_rng(24)
+    L, d = 290, 8
+    q, k, v = (_rand_bf16(rng, 1, 1, L, d) for _ in range(3))
+    bm = np.zeros((1, 1, 3, 3), np.uint8)
+    bm[0, 0, 2, 0] = 1                      # block 2 may see block 0
+    right = O.compressed_attention(q, k, v, np.array([L]), block_mask=bm)
+    wrong = O.compressed_attention(q, k, v, np.array([L]), block_mask=bm.transpose(0, 1, 3, 2).copy())
+    assert not np.allclose(right[0, 0, 256:], wrong[0, 0, 256:])
