@@ -235,6 +235,21 @@ tsa_status tsa_attend_gathered(const tsa_params* p, const void* q, const void* k
                                const int32_t* idx, const int32_t* k_seq, void* o, float* lse,
                                void* ws, size_t ws_bytes, void* stream);
 
+/* Steps 5(-6) with a block-sparse mask over the compressed sequence.  [GS]
+ * section 4 presents the method as complementary to block-sparse attention
+ * kernels (e.g. FlexPrefill): those run on the compressed tensors.  Same as
+ * tsa_attend (idx NULL: compressed output oc in o) or tsa_attend_scatter
+ * (idx given: output scattered into o in p->layout, other rows zero), except
+ * that compressed row i attends key j <= i only when j / 128 == i / 128 or
+ * block_mask[b, h, i / 128, j / 128] is nonzero.  block_mask: DEVICE uint8
+ * [B, Hq, NB, NB], NB = ceil(L / 128), caller-owned; entries above the
+ * diagonal are ignored and diagonal blocks are always attended.  KV tiles
+ * that neither query tile of a CTA's pair attends are skipped.
+ * ws: stage size. */
+tsa_status tsa_attend_blocks(const tsa_params* p, const void* qc, const void* kc, const void* vc,
+                             const int32_t* idx, const int32_t* k_seq, const uint8_t* block_mask, void* o,
+                             float* lse, void* ws, size_t ws_bytes, void* stream);
+
 /* Dense causal GQA attention on the uncompressed tensors (the baseline the
  * method is measured against; the same kernel as tsa_attend with the
  * identity selection): o[b,h,i] = sum_{j<=i} softmax_j(scale *
@@ -258,6 +273,19 @@ tsa_status tsa_scatter(const tsa_params* p, const void* oc, const int32_t* idx, 
 tsa_status tsa_forward(const tsa_params* p, const void* q, const void* k, const void* v, void* o,
                        float* scores_out, int32_t* idx_out, int32_t* k_seq_out,
                        void* ws, size_t ws_bytes, void* stream);
+
+/* Layer-level switch.  [GS] section 2 "Seleccion de Capas Dispersas" applies
+ * the method only in the layers chosen by a criterion on the model's hidden
+ * states (inter-layer representation drift); that criterion needs a model
+ * and is not computed here.  The caller supplies the choice instead:
+ * sparse_layers is a HOST array of n_layers flags (nonzero = sparse), and
+ * layer (0 <= layer < n_layers) selects this call's layer.  A sparse layer
+ * runs tsa_forward (same arguments and workspace rules); a dense layer runs
+ * tsa_attend_dense on q, k, v into o and leaves scores_out, idx_out and
+ * k_seq_out untouched.  ws: >= tsa_workspace_size bytes. */
+tsa_status tsa_layer_forward(const tsa_params* p, int32_t layer, const uint8_t* sparse_layers, int32_t n_layers,
+                             const void* q, const void* k, const void* v, void* o, float* scores_out,
+                             int32_t* idx_out, int32_t* k_seq_out, void* ws, size_t ws_bytes, void* stream);
 
 /* Proxy scores with no device allocation at all.  No counterpart on the
  * pages: an addition for callers that cannot call cudaMalloc (a plug-in whose

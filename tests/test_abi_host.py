@@ -121,6 +121,24 @@ def test_null_and_misaligned_pointers_rejected(lib):
     assert _call(lib, "tsa_get_device_status", None, None, None) == INVALID
 
 
+def test_layer_switch_arguments(lib):
+    p = ctypes.byref(good())
+    big = T.workspace_size(good())
+    flags = (ctypes.c_uint8 * 4)(1, 0, 1, 0)
+    fl = ctypes.cast(flags, ctypes.c_void_p)
+    args = (FAKE, FAKE, FAKE, FAKE, None, None, None, FAKE, big, None)
+    assert _call(lib, "tsa_layer_forward", p, 0, None, 4, *args) == INVALID      # no layer list
+    assert _call(lib, "tsa_layer_forward", p, 4, fl, 4, *args) == INVALID        # layer out of range
+    assert _call(lib, "tsa_layer_forward", p, -1, fl, 4, *args) == INVALID
+    assert _call(lib, "tsa_layer_forward", p, 0, fl, 0, *args) == INVALID        # empty list
+    # each branch reaches its own validation: sparse needs the full workspace,
+    # dense only the stage workspace
+    small = (FAKE, FAKE, FAKE, FAKE, None, None, None, FAKE, T.stage_workspace_size(good()), None)
+    assert _call(lib, "tsa_layer_forward", p, 0, fl, 4, *small) == WORKSPACE
+    assert _call(lib, "tsa_layer_forward", p, 1, fl, 4, FAKE, FAKE, None, FAKE, None, None, None, FAKE,
+                 big, None) == INVALID                                          # dense branch: null v
+
+
 def test_per_head_budget_needs_head_counts(lib):
     p = ctypes.byref(good(budget_mode="per_head"))
     ws_n = T.stage_workspace_size(good(budget_mode="per_head"))

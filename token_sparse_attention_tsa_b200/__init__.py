@@ -33,7 +33,8 @@ LAYOUTS = {"bhld": LAYOUT_BHLD, "blhd": LAYOUT_BLHD}
 EXPORTED = ("tsa_abi_version", "tsa_status_string", "tsa_check_params", "tsa_workspace_size",
             "tsa_stage_workspace_size", "tsa_reset_device_status", "tsa_get_device_status",
             "tsa_score", "tsa_budget", "tsa_select", "tsa_gather_qkv", "tsa_attend",
-            "tsa_attend_dense", "tsa_attend_scatter", "tsa_attend_gathered", "tsa_scatter", "tsa_forward", "tsa_score_noalloc")
+            "tsa_attend_dense", "tsa_attend_scatter", "tsa_attend_gathered", "tsa_attend_blocks", "tsa_scatter",
+            "tsa_forward", "tsa_layer_forward", "tsa_score_noalloc")
 
 
 class TSAError(RuntimeError):
@@ -109,8 +110,11 @@ def load(path: str | None = None):
             "tsa_attend_dense": ([_P, _v, _v, _v, _v, _v, _v, _sz, _v], ctypes.c_int),
             "tsa_attend_gathered": ([_P, _v, _v, _v, _v, _v, _v, _v, _v, _sz, _v], ctypes.c_int),
             "tsa_attend_scatter": ([_P, _v, _v, _v, _v, _v, _v, _v, _v, _sz, _v], ctypes.c_int),
+            "tsa_attend_blocks": ([_P, _v, _v, _v, _v, _v, _v, _v, _v, _v, _sz, _v], ctypes.c_int),
             "tsa_scatter": ([_P, _v, _v, _v, _v, _v, _sz, _v], ctypes.c_int),
             "tsa_forward": ([_P, _v, _v, _v, _v, _v, _v, _v, _v, _sz, _v], ctypes.c_int),
+            "tsa_layer_forward": ([_P, ctypes.c_int32, _v, ctypes.c_int32, _v, _v, _v, _v, _v, _v, _v, _v, _sz, _v],
+                                  ctypes.c_int),
             "tsa_score_noalloc": ([_P, _v, _v, _v, _v], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
@@ -268,6 +272,17 @@ def tsa_attend_scatter(p, qc, kc, vc, idx, k_seq, o, lse, ws, stream=None):
                                      _nbytes(ws), _stream(stream)), "tsa_attend_scatter")
 
 
+def tsa_attend_blocks(p, qc, kc, vc, idx, k_seq, block_mask, o, lse, ws, stream=None):
+    """idx None: compressed output in o; else o in the caller's layout."""
+    import torch
+    bf = torch.bfloat16
+    _check(load().tsa_attend_blocks(ctypes.byref(p), _ptr(qc, "qc", bf), _ptr(kc, "kc", bf), _ptr(vc, "vc", bf),
+                                    _ptr(idx, "idx", torch.int32), _ptr(k_seq, "k_seq", torch.int32),
+                                    _ptr(block_mask, "block_mask", torch.uint8), _ptr(o, "o", bf),
+                                    _ptr(lse, "lse", torch.float32), _ptr(ws, "ws"), _nbytes(ws),
+                                    _stream(stream)), "tsa_attend_blocks")
+
+
 def tsa_attend_gathered(p, q, k, v, idx, k_seq, o, lse, ws, stream=None):
     import torch
     bf = torch.bfloat16
@@ -292,6 +307,21 @@ def tsa_forward(p, q, k, v, o, ws, scores_out=None, idx_out=None, k_seq_out=None
                               _ptr(o, "o", bf), _ptr(scores_out, "scores_out", torch.float32),
                               _ptr(idx_out, "idx_out", torch.int32), _ptr(k_seq_out, "k_seq_out", torch.int32),
                               _ptr(ws, "ws"), _nbytes(ws), _stream(stream)), "tsa_forward")
+
+
+def tsa_layer_forward(p, layer: int, sparse_layers, q, k, v, o, ws, scores_out=None, idx_out=None, k_seq_out=None,
+                      stream=None):
+    """sparse_layers: a sequence of per-layer flags (host side), e.g. a list
+    of bools; layer selects this call's entry."""
+    import torch
+    bf = torch.bfloat16
+    flags = (ctypes.c_uint8 * len(sparse_layers))(*[1 if x else 0 for x in sparse_layers])
+    _check(load().tsa_layer_forward(ctypes.byref(p), int(layer), ctypes.cast(flags, ctypes.c_void_p),
+                                    len(sparse_layers), _ptr(q, "q", bf), _ptr(k, "k", bf), _ptr(v, "v", bf),
+                                    _ptr(o, "o", bf), _ptr(scores_out, "scores_out", torch.float32),
+                                    _ptr(idx_out, "idx_out", torch.int32),
+                                    _ptr(k_seq_out, "k_seq_out", torch.int32), _ptr(ws, "ws"), _nbytes(ws),
+                                    _stream(stream)), "tsa_layer_forward")
 
 
 def forward(q, k, v, w: int, tau: float, softmax_scale: float = 0.0, ws=None, return_intermediates=False,

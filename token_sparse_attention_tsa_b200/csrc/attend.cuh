@@ -42,6 +42,8 @@ struct AttnArgs {
   int token_major;        // Q/K/V maps are (d, H, L, B) (else (d, L, H, B)); gather rows likewise
   int in_packed;          // Q/K/V are packed sequences (token coordinate cu[b] + t, one map "sequence")
   Seqs seqs;              // sequence lengths L_b (and packed token offsets)
+  const uint8_t* block_mask;  // [B*Hq, n_tiles, n_tiles] or null: query tile i may attend key tile j
+                              // (j < i) only where the entry is nonzero; diagonal tiles always
 };
 
 // ---------------------------------------------------------------------------
@@ -107,7 +109,9 @@ struct Attn2Layout {
 // pass before the kernel is faster when compressed buffers can be held.)
 // kScatter: output row i is written to row idx[i] of o (in place in the
 // full-length output) instead of row i of a compressed output.
-template <int D, bool kGather, bool kScatter>
+// kBlocks: KV tiles are filtered by the block mask (without it every tile
+// in the causal range is processed and the checks compile away).
+template <int D, bool kGather, bool kScatter, bool kBlocks = false>
 __global__ void __launch_bounds__(Attn2Layout<D>::THREADS, 1)
     attend2_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, const AttnArgs a) {
@@ -130,6 +134,20 @@ __global__ void __launch_bounds__(Attn2Layout<D>::THREADS, 1)
   const bool two = (t0 + 1) * C::BM < valid;       // second query tile has rows
   const int last0 = t0;                            // tile 0 attends KV tiles 0..t0
   const int n_kv = two ? t0 + 2 : t0 + 1;          // tile 1 attends 0..t0+1
+
+  // KV tiles this CTA processes: those one of its query tiles attends (its
+  // causal range, the diagonal always, earlier tiles where the block mask
+  // allows).  Producer, MMA issuer and softmax walk the same list; barrier
+  // phases and ring slots count processed tiles, not j.
+  const uint8_t* bmask = kBlocks ? a.block_mask + static_cast<size_t>(bh) * a.n_tiles * a.n_tiles : nullptr;
+  auto needs = [&](int qt, int j) {
+    if constexpr (kBlocks) return j <= qt && (j == qt || __ldg(bmask + static_cast<size_t>(qt) * a.n_tiles + j) != 0);
+    return j <= qt;
+  };
+  auto proc = [&](int j) {
+    if constexpr (kBlocks) return needs(t0, j) || (two && needs(t0 + 1, j));
+    return true;                                 // every j < n_kv
+  };
 
   auto bar = [&](int i) -> uint32_t { return base + C::OFF_BAR + 8u * static_cast<uint32_t>(i); };
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(gbase + C::OFF_BAR + 8 * C::B_COUNT);
@@ -216,14 +234,22 @@ __global__ void __launch_bounds__(Attn2Layout<D>::THREADS, 1)
       load_tile(q_by_index, base + C::OFF_Q0, &tmQ, bar(C::B_Q), t0, h, a.Hq);
       if (two) load_tile(q_by_index, base + C::OFF_Q1, &tmQ, bar(C::B_Q), t0 + 1, h, a.Hq);
       int issued = 0;
-      for (int n = 0; n < 2 * n_kv; ++n) {
-        const int s = slot_of(n), u = use_of(n);
-        if (u >= 1 && !__all_sync(0xffffffffu, mbar_wait(bar(C::B_EMPTY + s), (u - 1) & 1, wc))) break;
-        if (leader) mbar_arrive_expect_tx(bar(C::B_FULL + s), C::TILE);
-        __syncwarp();
-        load_tile(kv_by_index, ring(n), (n & 1) ? &tmV : &tmK, bar(C::B_FULL + s), n >> 1, h / a.G_map,
-                  a.Hkv_map);
-        issued = n + 1;
+      bool go = true;
+      for (int j = 0, cb = 0; go && j < n_kv; ++j) {
+        if (!proc(j)) continue;
+        const int c = kBlocks ? cb++ : j;      // processed-tile count (j itself without a mask)
+        for (int kv = 0; kv < 2; ++kv) {        // K_j, V_j into ring positions 2c, 2c+1
+          const int n = 2 * c + kv;
+          const int s = slot_of(n), u = use_of(n);
+          if (u >= 1 && !__all_sync(0xffffffffu, mbar_wait(bar(C::B_EMPTY + s), (u - 1) & 1, wc))) {
+            go = false;
+            break;
+          }
+          if (leader) mbar_arrive_expect_tx(bar(C::B_FULL + s), C::TILE);
+          __syncwarp();
+          load_tile(kv_by_index, ring(n), kv ? &tmV : &tmK, bar(C::B_FULL + s), j, h / a.G_map, a.Hkv_map);
+          issued = n + 1;
+        }
       }
       if (leader && *cta_abort) {  // let every copy still in flight land before exit
         mbar_wait_drain(bar(C::B_Q), 0, 1000000000ull);
@@ -246,9 +272,9 @@ __global__ void __launch_bounds__(Attn2Layout<D>::THREADS, 1)
       const uint64_t dq1 = smem_desc(base + C::OFF_Q1, 16, 1024, kSwizzle128B);
       const uint64_t dk0 = smem_desc(base + C::OFF_RING, 16, 1024, kSwizzle128B);
       const uint64_t dv0 = smem_desc(base + C::OFF_RING, C::CHUNK, 1024, kSwizzle128B);
-      auto issue_s = [&](int t, int j) {
+      auto issue_s = [&](int t, int c) {         // c: processed-tile count of the KV tile
         const uint64_t dq = t ? dq1 : dq0;
-        const uint64_t dk = dk0 + static_cast<uint64_t>((slot_of(2 * j) * C::TILE) >> 4);
+        const uint64_t dk = dk0 + static_cast<uint64_t>((slot_of(2 * c) * C::TILE) >> 4);
         if (leader) {
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
@@ -267,18 +293,18 @@ __global__ void __launch_bounds__(Attn2Layout<D>::THREADS, 1)
       auto full = [&](int n) { return wait_all(bar(C::B_FULL + slot_of(n)), use_of(n) & 1); };
       // O_t += P_t,j V_j, one group of k-steps per released P group.  P of
       // keys [16kk, 16kk+16) sits in TMEM column 8kk of the tile's S columns.
-      auto issue_pv = [&](int t, int j) -> bool {
-        const uint64_t dv = dv0 + static_cast<uint64_t>((slot_of(2 * j + 1) * C::TILE) >> 4);
+      auto issue_pv = [&](int t, int c) -> bool {
+        const uint64_t dv = dv0 + static_cast<uint64_t>((slot_of(2 * c + 1) * C::TILE) >> 4);
         constexpr int KPG = C::KSTEPS / C::P_SPLITS;
 #pragma unroll
         for (int g = 0; g < C::P_SPLITS; ++g) {
-          if (!wait_all(bar(C::B_P + t * C::P_SPLITS + g), j & 1)) return false;
+          if (!wait_all(bar(C::B_P + t * C::P_SPLITS + g), c & 1)) return false;
           tc_fence_after();
           if (leader) {
 #pragma unroll
             for (int kk = g * KPG; kk < (g + 1) * KPG; ++kk)
               mma_bf16_ts(tmem + C::TMEM_O + t * D, tmem + t * 128 + 8 * kk,
-                          dv + static_cast<uint64_t>((kk * 2048) >> 4), idO, (j > 0 || kk > 0) ? 1u : 0u);
+                          dv + static_cast<uint64_t>((kk * 2048) >> 4), idO, (c > 0 || kk > 0) ? 1u : 0u);
           }
         }
         commit_to(bar(C::B_PV + t));
@@ -291,29 +317,36 @@ __global__ void __launch_bounds__(Attn2Layout<D>::THREADS, 1)
       // them here cannot deadlock the ring.
       // test hook: phase 0 of the drain barrier completes only at teardown,
       // so this bounded wait runs out and takes the abort path
+      int n_proc = n_kv;
+      if constexpr (kBlocks) {
+        n_proc = 0;
+        for (int j = 0; j < n_kv; ++j) n_proc += proc(j) ? 1 : 0;   // >= 1: tile 0's diagonal
+      }
       bool ok = !(a.test_stall && !wait_all(bar(C::B_DRAIN), 0)) && wait_all(bar(C::B_Q), 0) && full(0);
-      for (int j = 0; ok && j < n_kv; ++j) {
-        tc_fence_after();                                                // K_j has landed
-        if (j <= last0) issue_s(0, j);
-        if (two && j >= 1) {
-          if (!(ok = issue_pv(1, j - 1))) break;
-          commit_to(bar(C::B_EMPTY + slot_of(2 * j - 1)));               // V_{j-1} done
+      for (int j = 0, cb = 0; ok && j < n_kv; ++j) {
+        if (!proc(j)) continue;
+        const int c = kBlocks ? cb++ : j;        // processed-tile count (j itself without a mask)
+        tc_fence_after();                                                // K of tile c has landed
+        if (j <= last0) issue_s(0, c);
+        if (two && c >= 1) {
+          if (!(ok = issue_pv(1, c - 1))) break;
+          commit_to(bar(C::B_EMPTY + slot_of(2 * c - 1)));               // V of tile c-1 done
         }
-        if (two) issue_s(1, j);
-        commit_to(bar(C::B_EMPTY + slot_of(2 * j)));                     // K_j done
-        const bool more = j + 1 < n_kv;
+        if (two) issue_s(1, c);
+        commit_to(bar(C::B_EMPTY + slot_of(2 * c)));                     // K of tile c done
+        const bool more = c + 1 < n_proc;
         if (j <= last0) {
-          if (!(ok = full(2 * j + 1))) break;                            // V_j
-          if (more && !(ok = full(2 * j + 2))) break;                    // K_{j+1}
-          if (!(ok = issue_pv(0, j))) break;
-          if (!two) commit_to(bar(C::B_EMPTY + slot_of(2 * j + 1)));
-        } else if (more && !(ok = full(2 * j + 2))) {
+          if (!(ok = full(2 * c + 1))) break;                            // V of tile c
+          if (more && !(ok = full(2 * c + 2))) break;                    // K of tile c+1
+          if (!(ok = issue_pv(0, c))) break;
+          if (!two) commit_to(bar(C::B_EMPTY + slot_of(2 * c + 1)));
+        } else if (more && !(ok = full(2 * c + 2))) {
           break;
         }
       }
       if (ok && two) {
-        const int j = n_kv - 1;
-        if (full(2 * j + 1) && issue_pv(1, j)) commit_to(bar(C::B_EMPTY + slot_of(2 * j + 1)));
+        const int c = n_proc - 1;
+        if (full(2 * c + 1) && issue_pv(1, c)) commit_to(bar(C::B_EMPTY + slot_of(2 * c + 1)));
       }
       commit_to(bar(C::B_DRAIN));
       if (leader) mbar_wait_drain(bar(C::B_DRAIN), 0, 1000000000ull);
@@ -334,9 +367,28 @@ __global__ void __launch_bounds__(Attn2Layout<D>::THREADS, 1)
     float m_used = -INFINITY;
     float l = 0.f;
     bool live = true;
+    int pc = -1;                                 // processed-tile count of the current KV tile
     for (int j = 0; j <= last; ++j) {
-      if (!(live = __all_sync(0xffffffffu, mbar_wait(bar(C::B_S + tt), j & 1, wc)))) break;
+      if (!proc(j)) continue;
+      pc = kBlocks ? pc + 1 : j;
+      if (!(live = __all_sync(0xffffffffu, mbar_wait(bar(C::B_S + tt), pc & 1, wc)))) break;
       tc_fence_after();
+      if (kBlocks && !needs(tile, j)) {
+        // a tile only the other query tile attends: P = 0 (S is not read)
+        uint32_t z[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) z[e] = 0u;
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) tmem_st16u(s_col + cc * 16, z);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+#pragma unroll
+          for (int g = 0; g < C::P_SPLITS; ++g) mbar_arrive(bar(C::B_P + tt * C::P_SPLITS + g));
+        }
+        continue;
+      }
       const bool diag = (j == last);
       float sv[4][32];
 #pragma unroll
@@ -395,8 +447,8 @@ __global__ void __launch_bounds__(Attn2Layout<D>::THREADS, 1)
           // PV barrier can never be two phases ahead here because P.V j
           // needs this tile's P first, so a parity wait after skipped ones
           // still names the right phase.
-          if (j > 0 && __any_sync(0xffffffffu, resc)) {
-            if (!(live = __all_sync(0xffffffffu, mbar_wait(bar(C::B_PV + tt), (j - 1) & 1, wc)))) break;
+          if (pc > 0 && __any_sync(0xffffffffu, resc)) {
+            if (!(live = __all_sync(0xffffffffu, mbar_wait(bar(C::B_PV + tt), (pc - 1) & 1, wc)))) break;
             tc_fence_after();
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
@@ -409,7 +461,7 @@ __global__ void __launch_bounds__(Attn2Layout<D>::THREADS, 1)
             }
           }
           if (diag && last_active && (j * C::BN + C::BN > valid)) {
-            const int n = 2 * j + 1;
+            const int n = 2 * pc + 1;                // ring position of this tile's V
             if (!(live = __all_sync(0xffffffffu, mbar_wait(bar(C::B_FULL + slot_of(n)), use_of(n) & 1, wc)))) break;
             if (j * C::BN + r >= valid) {
 #pragma unroll
@@ -436,7 +488,7 @@ __global__ void __launch_bounds__(Attn2Layout<D>::THREADS, 1)
       l = l * alpha + (((rs[0] + rs[1]) + (rs[2] + rs[3])) + ((rs[4] + rs[5]) + (rs[6] + rs[7])));
     }
     // ------------------------------------------------------------ epilogue
-    live = live && __all_sync(0xffffffffu, mbar_wait(bar(C::B_PV + tt), last & 1, wc));
+    live = live && __all_sync(0xffffffffu, mbar_wait(bar(C::B_PV + tt), pc & 1, wc));
     if (live) {
       tc_fence_after();
       const float inv_l = 1.f / l;

@@ -181,7 +181,8 @@ bool ensure_smem(std::atomic<int> (&done)[kMaxDevices], K kernel, int bytes) {
 std::atomic<int> g_attn64[kMaxDevices], g_attn128[kMaxDevices], g_gath64[kMaxDevices], g_gath128[kMaxDevices],
     g_gq64[kMaxDevices], g_gq128[kMaxDevices], g_st64[kMaxDevices],
     g_st128[kMaxDevices], g_sum64[kMaxDevices], g_sum128[kMaxDevices], g_budget[kMaxDevices],
-    g_select[kMaxDevices];
+    g_select[kMaxDevices], g_blk64[kMaxDevices], g_blk128[kMaxDevices], g_blks64[kMaxDevices],
+    g_blks128[kMaxDevices];
 
 constexpr int kBudgetSmem = tsa::BS_WARPS * 256 * (8 + 4);
 constexpr int kSelectSmem = tsa::BS_WARPS * 256 * 4;
@@ -325,7 +326,7 @@ tsa_status run_scatter(const tsa_params* p, const void* oc, const int32_t* idx, 
 tsa_status run_attend(const tsa_params* p, const void* q, const void* k, const void* v, int heads_kv, int g_kv,
                       const int32_t* k_seq, void* o, float* lse, uint32_t* status, uint32_t* abort_word,
                       cudaStream_t st, bool in_caller, bool out_caller, const int32_t* idx = nullptr,
-                      bool gather = false) {
+                      bool gather = false, const uint8_t* block_mask = nullptr) {
   CUtensorMap mq, mk, mv;
   const bool scatter = idx != nullptr;
   gather = gather && scatter;
@@ -359,6 +360,7 @@ tsa_status run_attend(const tsa_params* p, const void* q, const void* k, const v
   a.in_packed = (in_caller && packed(p)) ? 1 : 0;
   a.seqs = seqs_of(p);
   a.os = out_caller ? caller_strides(p, p->Hq) : strides_of(false, p->Hq, p->L, p->d);
+  a.block_mask = block_mask;
   const dim3 grid((a.n_tiles + 1) / 2, p->B * p->Hq);  // two query tiles per CTA
   auto launch = [&](auto kernel, std::atomic<int>(&attr)[kMaxDevices], int threads, int smem) -> tsa_status {
     if (!ensure_smem(attr, kernel, smem)) return TSA_ERR_CUDA;
@@ -367,11 +369,19 @@ tsa_status run_attend(const tsa_params* p, const void* q, const void* k, const v
   };
   if (p->d == 128) {
     using L = tsa::Attn2Layout<128>;
+    if (block_mask) {
+      if (!scatter) return launch(tsa::attend2_kernel<128, false, false, true>, g_blk128, L::THREADS, L::ALLOC);
+      return launch(tsa::attend2_kernel<128, false, true, true>, g_blks128, L::THREADS, L::ALLOC);
+    }
     if (!scatter) return launch(tsa::attend2_kernel<128, false, false>, g_attn128, L::THREADS, L::ALLOC);
     if (!gather) return launch(tsa::attend2_kernel<128, false, true>, g_gq128, L::THREADS, L::ALLOC);
     return launch(tsa::attend2_kernel<128, true, true>, g_gath128, L::THREADS, L::ALLOC);
   }
   using L = tsa::Attn2Layout<64>;
+  if (block_mask) {
+    if (!scatter) return launch(tsa::attend2_kernel<64, false, false, true>, g_blk64, L::THREADS, L::ALLOC);
+    return launch(tsa::attend2_kernel<64, false, true, true>, g_blks64, L::THREADS, L::ALLOC);
+  }
   if (!scatter) return launch(tsa::attend2_kernel<64, false, false>, g_attn64, L::THREADS, L::ALLOC);
   if (!gather) return launch(tsa::attend2_kernel<64, false, true>, g_gq64, L::THREADS, L::ALLOC);
   return launch(tsa::attend2_kernel<64, true, true>, g_gath64, L::THREADS, L::ALLOC);
@@ -614,6 +624,33 @@ tsa_status tsa_attend_gathered(const tsa_params* p, const void* q, const void* k
                       true, idx, true)) != TSA_OK)
     return s;
   return run_zero_unselected(p, idx, k_seq, o, status_of(ws), st);
+}
+
+tsa_status tsa_attend_blocks(const tsa_params* p, const void* qc, const void* kc, const void* vc,
+                             const int32_t* idx, const int32_t* k_seq, const uint8_t* block_mask, void* o,
+                             float* lse, void* ws, size_t ws_bytes, void* stream) {
+  tsa_status s = tsa_check_params(p);
+  if (s != TSA_OK) return s;
+  if (!tensors_ok({qc, kc, vc, k_seq, o}) || !block_mask || (idx && !aligned(idx, 16)) ||
+      (lse && !aligned(lse, 4)))
+    return TSA_ERR_INVALID_ARG;
+  if ((s = check_ws(p, ws, ws_bytes, false)) != TSA_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if ((s = run_attend(p, qc, kc, vc, p->Hq, 1, k_seq, o, lse, status_of(ws), abort_of(ws), st, false,
+                      idx != nullptr, idx, false, block_mask)) != TSA_OK)
+    return s;
+  return idx ? run_zero_unselected(p, idx, k_seq, o, status_of(ws), st) : TSA_OK;
+}
+
+tsa_status tsa_layer_forward(const tsa_params* p, int32_t layer, const uint8_t* sparse_layers, int32_t n_layers,
+                             const void* q, const void* k, const void* v, void* o, float* scores_out,
+                             int32_t* idx_out, int32_t* k_seq_out, void* ws, size_t ws_bytes, void* stream) {
+  tsa_status s = tsa_check_params(p);
+  if (s != TSA_OK) return s;
+  if (!sparse_layers || n_layers < 1 || layer < 0 || layer >= n_layers) return TSA_ERR_INVALID_ARG;
+  if (sparse_layers[layer])
+    return tsa_forward(p, q, k, v, o, scores_out, idx_out, k_seq_out, ws, ws_bytes, stream);
+  return tsa_attend_dense(p, q, k, v, o, nullptr, ws, ws_bytes, stream);
 }
 
 }  // extern "C"
