@@ -405,6 +405,33 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
     except Exception:
         sdpa_ms = None
 
+    # ---- optional: block-sparse composition on the compressed sequence
+    blocks = None
+    if args.blocks:
+        nbw = int(args.blocks.split(":")[1])
+        nb = (wl.L + 127) // 128
+        ii = torch.arange(nb, device=dev)[:, None]
+        jj = torch.arange(nb, device=dev)[None, :]
+        band = (((ii - jj) <= nbw) | (jj == 0)) & (jj <= ii)
+        bmask = band.to(torch.uint8).expand(wl.B, wl.Hq, nb, nb).contiguous()
+
+        def blocks_fwd():
+            T.tsa_score(p, q, k, scores, ws)
+            T.tsa_budget(p, scores, k_head, k_seq, ws)
+            T.tsa_select(p, scores, kept, idx, ws)
+            T.tsa_gather_qkv(p, q, k, v, idx, kept, qc, kc, vc, ws)
+            T.tsa_attend_blocks(p, qc, kc, vc, idx, kept, bmask, o, None, ws)
+
+        for _ in range(2):
+            blocks_fwd()
+        bms = timed(blocks_fwd, max(2, args.steps // 2))
+        kb_rows = ks[0]
+        nbk = (kb_rows + 127) // 128
+        frac = float(band[:nbk, :nbk].sum().item()) / (nbk * (nbk + 1) / 2)
+        blocks = {"mask": f"sink block + local band of {nbw} blocks (128 compressed tokens each)",
+                  "ms_per_step": bms, "effective_tflops": dense_flops(wl) / (bms * 1e-3) / 1e12,
+                  "causal_tile_fraction_kept": frac, "speedup_vs_tsa": ms / bms}
+
     # ---- end to end: pinned host inputs -> device -> tsa_forward -> host output
     o_host = torch.empty(tuple(o.shape), dtype=torch.bfloat16).pin_memory()
 
@@ -475,6 +502,8 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": KERNELS_PER_FORWARD * args.steps, "clocks": clocks,
     }
+    if blocks is not None:
+        line["block_sparse"] = blocks
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:
@@ -495,6 +524,9 @@ def main() -> int:
     ap.add_argument("--budget-mode", default="max", choices=["max", "mean", "per_head"])
     ap.add_argument("--keep-recent", type=int, default=0)
     ap.add_argument("--layout", default="bhld", choices=["bhld", "blhd"])
+    ap.add_argument("--blocks", default=None,
+                    help="band:N -- also time the path with a block-sparse mask on the compressed sequence "
+                         "(sink block + local band of N blocks)")
     ap.add_argument("--varlen", default=None,
                     help="comma-separated sequence lengths: time a packed varlen batch of the workload's "
                          "first L_b tokens per sequence instead of the headline step")

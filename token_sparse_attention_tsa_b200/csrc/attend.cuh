@@ -85,7 +85,9 @@ struct Attn2Layout {
   static constexpr int OFF_Q1 = TILE;
   static constexpr int OFF_RING = 2 * TILE;
   static constexpr int OFF_BAR = OFF_RING + NSLOT * TILE;
-  static constexpr int TOTAL = OFF_BAR + 512;
+  static constexpr int OFF_PROC = OFF_BAR + 512;      // bit j: KV tile j is processed (block masks)
+  static constexpr int MAX_TILES = 32768;             // L <= 2^22 tokens
+  static constexpr int TOTAL = OFF_PROC + MAX_TILES / 8;
   static constexpr int ALLOC = (TOTAL + 1024) > 120 * 1024 ? (TOTAL + 1024) : 120 * 1024;
   static constexpr int TMEM_COLS = 512;
   static constexpr int TMEM_O = 256;
@@ -144,9 +146,20 @@ __global__ void __launch_bounds__(Attn2Layout<D>::THREADS, 1)
     if constexpr (kBlocks) return j <= qt && (j == qt || __ldg(bmask + static_cast<size_t>(qt) * a.n_tiles + j) != 0);
     return j <= qt;
   };
-  auto proc = [&](int j) {
-    if constexpr (kBlocks) return needs(t0, j) || (two && needs(t0 + 1, j));
-    return true;                                 // every j < n_kv
+  // With a block mask the CTA's processed tiles are computed once into a
+  // shared bitmask (below); next_proc(j) is the first processed tile >= j
+  // (n_kv when none is left).  Without one every tile is processed.
+  const uint32_t* proc_bits = reinterpret_cast<const uint32_t*>(gbase + C::OFF_PROC);
+  auto next_proc = [&](int j) -> int {
+    if constexpr (kBlocks) {
+      while (j < n_kv) {
+        const uint32_t w = proc_bits[j >> 5] >> (j & 31);
+        if (w) return j + __ffs(static_cast<int>(w)) - 1;
+        j = (j | 31) + 1;
+      }
+      return n_kv;
+    }
+    return j;
   };
 
   auto bar = [&](int i) -> uint32_t { return base + C::OFF_BAR + 8u * static_cast<uint32_t>(i); };
@@ -170,6 +183,15 @@ __global__ void __launch_bounds__(Attn2Layout<D>::THREADS, 1)
     mbar_init(bar(C::B_DRAIN), 1);
     *cta_abort = (a.abort_word && *reinterpret_cast<volatile uint32_t*>(a.abort_word)) ? 1 : 0;
     fence_mbar_init();
+  }
+  if constexpr (kBlocks) {  // processed tiles: one of the pair's query tiles attends them
+    uint32_t* bits = reinterpret_cast<uint32_t*>(gbase + C::OFF_PROC);
+    for (int w = warp; w * 32 < n_kv; w += C::THREADS / 32) {
+      const int j = w * 32 + lane;
+      const bool pj = j < n_kv && (needs(t0, j) || (two && needs(t0 + 1, j)));
+      const uint32_t word = __ballot_sync(0xffffffffu, pj);
+      if (lane == 0) bits[w] = word;
+    }
   }
   if (warp == C::MMA_WARP) {
     tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
@@ -235,8 +257,7 @@ __global__ void __launch_bounds__(Attn2Layout<D>::THREADS, 1)
       if (two) load_tile(q_by_index, base + C::OFF_Q1, &tmQ, bar(C::B_Q), t0 + 1, h, a.Hq);
       int issued = 0;
       bool go = true;
-      for (int j = 0, cb = 0; go && j < n_kv; ++j) {
-        if (!proc(j)) continue;
+      for (int j = next_proc(0), cb = 0; go && j < n_kv; j = next_proc(j + 1)) {
         const int c = kBlocks ? cb++ : j;      // processed-tile count (j itself without a mask)
         for (int kv = 0; kv < 2; ++kv) {        // K_j, V_j into ring positions 2c, 2c+1
           const int n = 2 * c + kv;
@@ -320,11 +341,10 @@ __global__ void __launch_bounds__(Attn2Layout<D>::THREADS, 1)
       int n_proc = n_kv;
       if constexpr (kBlocks) {
         n_proc = 0;
-        for (int j = 0; j < n_kv; ++j) n_proc += proc(j) ? 1 : 0;   // >= 1: tile 0's diagonal
+        for (int w = 0; w * 32 < n_kv; ++w) n_proc += __popc(proc_bits[w]);   // >= 1: tile 0's diagonal
       }
       bool ok = !(a.test_stall && !wait_all(bar(C::B_DRAIN), 0)) && wait_all(bar(C::B_Q), 0) && full(0);
-      for (int j = 0, cb = 0; ok && j < n_kv; ++j) {
-        if (!proc(j)) continue;
+      for (int j = next_proc(0), cb = 0; ok && j < n_kv; j = next_proc(j + 1)) {
         const int c = kBlocks ? cb++ : j;        // processed-tile count (j itself without a mask)
         tc_fence_after();                                                // K of tile c has landed
         if (j <= last0) issue_s(0, c);
@@ -368,8 +388,7 @@ __global__ void __launch_bounds__(Attn2Layout<D>::THREADS, 1)
     float l = 0.f;
     bool live = true;
     int pc = -1;                                 // processed-tile count of the current KV tile
-    for (int j = 0; j <= last; ++j) {
-      if (!proc(j)) continue;
+    for (int j = next_proc(0); j <= last; j = next_proc(j + 1)) {
       pc = kBlocks ? pc + 1 : j;
       if (!(live = __all_sync(0xffffffffu, mbar_wait(bar(C::B_S + tt), pc & 1, wc)))) break;
       tc_fence_after();
