@@ -36,12 +36,12 @@ import workloads as W  # noqa: E402
 METRIC = "Token-sparse prefill attention ms and effective TFLOP/s at 128K vs dense; % BF16/HBM roofline"
 UNIT = "TFLOP/s (effective: dense causal attention FLOPs / TSA time)"
 DEFAULT_WORKLOAD = "c4_L128K_gqa"
-KERNELS_PER_FORWARD = 8  # score x3, budget, select, gather, attention (scatter epilogue), zero fill
+KERNELS_PER_FORWARD = 9  # score x3, budget, budget finalize, select, gather, attention (scatter epilogue), zero fill
 # DRAM bytes per kept (head, row) of the attention kernel with the scatter
 # epilogue, from ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch
-# on the 32K workload (813.1 MB for 32 x 25147 kept rows); DRAM traffic grows
+# on the 32K workload (813.4 MB for 32 x 25147 kept rows); DRAM traffic grows
 # with kept rows, not with FLOPs (algorithmic: 3 x 256 B read + 256 B written).
-ATTN_DRAM_BYTES_PER_KEPT_ROW = 813.1e6 / (32 * 25147)
+ATTN_DRAM_BYTES_PER_KEPT_ROW = 813.4e6 / (32 * 25147)
 
 
 def dense_flops(wl) -> float:
