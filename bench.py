@@ -183,6 +183,14 @@ def oracle_sample(wl, tau: float, rows: int = 384, keep_recent: int = 0) -> dict
                        f"(of k={kh}); scaled by head count and by causal pair count to the full step")}
 
 
+def config_of(args, wl, world: int) -> dict:
+    """The workload description both arms print."""
+    return {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "L": wl.L, "d": wl.d, "w": wl.w,
+            "tau": args.tau, "budget_mode": args.budget_mode, "keep_recent": args.keep_recent,
+            "layout": args.layout, "parallelism": f"replicas{world}" if world > 1 else "single",
+            "l2": "inputs larger than L2 (Q 1 GiB, K/V 256 MiB each)"}
+
+
 def run_reference(args, wl, rank: int) -> int:
     if rank != 0:
         return 0
@@ -195,8 +203,7 @@ def run_reference(args, wl, rank: int) -> int:
         "metric": METRIC, "value": value, "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "L": wl.L, "d": wl.d,
-                   "w": wl.w, "tau": args.tau, "budget_mode": args.budget_mode, "keep_recent": args.keep_recent},
+        "config": config_of(args, wl, args.gpus),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": runs[0]["cores"], "kind": "oracle",
                          "sample": runs[0]["sample"]},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -517,11 +524,7 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "L": wl.L, "d": wl.d, "w": wl.w,
-                   "tau": args.tau, "budget_mode": args.budget_mode, "keep_recent": args.keep_recent,
-                   "layout": args.layout,
-                   "parallelism": f"replicas{world}" if world > 1 else "single",
-                   "l2": "inputs larger than L2 (Q 1 GiB, K/V 256 MiB each)"},
+        "config": config_of(args, wl, world),
         "k_seq": ks, "keep_fraction": [x / wl.L for x in ks],
         "kept_fraction_all_heads": kept_rows / float(wl.B * wl.Hq * wl.L),
         "dense_ms": dense_ms, "speedup_vs_dense": dense_ms / ms, "sdpa_dense_ms": sdpa_ms,
