@@ -420,14 +420,16 @@ __global__ void __launch_bounds__(Attn2Layout<D>::THREADS, 1)
           for (int e = 0; e < 32; ++e)
             if (c * 32 + e > r) sv[c][e] = -INFINITY;
       }
-      // row max: four chains of three-input maxima over value pairs
-      float m4[4] = {sv[0][0], sv[0][1], sv[0][2], sv[0][3]};
+      // row max: eight chains of three-input maxima over value pairs
+      float m8[8];
 #pragma unroll
-      for (int i = 4; i < C::BN; i += 2) {       // i even: i, i+1 lie in one 32-chunk
-        const int u = (i >> 1) & 3;
-        m4[u] = fmax3(m4[u], sv[i >> 5][i & 31], sv[i >> 5][(i & 31) + 1]);
+      for (int u = 0; u < 8; ++u) m8[u] = sv[0][u];
+#pragma unroll
+      for (int i = 8; i < C::BN; i += 2) {       // i even: i, i+1 lie in one 32-chunk
+        const int u = (i >> 1) & 7;
+        m8[u] = fmax3(m8[u], sv[i >> 5][i & 31], sv[i >> 5][(i & 31) + 1]);
       }
-      const float mx = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
+      const float mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
       const float m_new = fmaxf(m_used, mx * sl2);
       const bool resc = m_new > m_used + 8.0f;   // lazy rescale (factor <= 2^8 tolerated)
       const float alpha = resc ? ex2_approx(m_used - m_new) : 1.f;
@@ -438,14 +440,19 @@ __global__ void __launch_bounds__(Attn2Layout<D>::THREADS, 1)
 #pragma unroll
       for (int u = 0; u < 4; ++u) r4[u] = 0ull;
       // S columns [32c, 32c+32) give P columns [16c, 16c+16); every S value
-      // is already in registers, so P may overwrite any S column.
+      // is already in registers, so P may overwrite any S column.  The plain
+      // kernel stores a group's P (its two chunks, 32 columns) in one go; the
+      // scatter and block-mask variants (more registers live) chunk by chunk.
+      constexpr bool kWide = !kScatter && !kBlocks;
       constexpr int CPG = 4 / C::P_SPLITS;          // 32-column chunks per P group
+      static_assert(CPG == 2, "one 32-column P store per group");
 #pragma unroll
       for (int g = 0; g < C::P_SPLITS; ++g) {
+        uint32_t pk32[32];
 #pragma unroll
         for (int cc = 0; cc < CPG; ++cc) {
           const int c = g * CPG + cc;
-          uint32_t pk[16];
+          uint32_t (&pk)[16] = *reinterpret_cast<uint32_t(*)[16]>(&pk32[kWide ? cc * 16 : 0]);
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             float x0, x1;
@@ -455,8 +462,9 @@ __global__ void __launch_bounds__(Attn2Layout<D>::THREADS, 1)
             r4[e & 3] = f2_add(r4[e & 3], f2_pack(p0, p1));
             pk[e] = pack_bf16x2(p0, p1);
           }
-          tmem_st16u(s_col + c * 16, pk);
+          if constexpr (!kWide) tmem_st16u(s_col + c * 16, pk);
         }
+        if constexpr (kWide) tmem_st32(s_col + g * 32, *reinterpret_cast<float(*)[32]>(pk32));
         if (g == 0) {
           // Before the first P group is released: O is rescaled when a
           // row's max grew past the lazy threshold, and V rows past `valid`
