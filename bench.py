@@ -39,9 +39,9 @@ DEFAULT_WORKLOAD = "c4_L128K_gqa"
 KERNELS_PER_FORWARD = 9  # score x3, budget, budget finalize, select, gather, attention (scatter epilogue), zero fill
 # DRAM bytes per kept (head, row) of the attention kernel with the scatter
 # epilogue, from ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch
-# on the 32K workload (813.4 MB for 32 x 25147 kept rows); DRAM traffic grows
+# on the 32K workload (811.5 MB for 32 x 25147 kept rows); DRAM traffic grows
 # with kept rows, not with FLOPs (algorithmic: 3 x 256 B read + 256 B written).
-ATTN_DRAM_BYTES_PER_KEPT_ROW = 813.4e6 / (32 * 25147)
+ATTN_DRAM_BYTES_PER_KEPT_ROW = 811.5e6 / (32 * 25147)
 
 
 def dense_flops(wl) -> float:
@@ -496,7 +496,7 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
     cflops = compressed_flops(wl, kept_np)
     attn_ms = stage_ms["attend"]
     achieved = cflops / (attn_ms * 1e-3) / 1e12
-    roof = {"bound": "tensor", "kernel": "attend2_kernel<128,false,true> (attention + scatter epilogue)",
+    roof = {"bound": "tensor", "kernel": "attend2_kernel<128,false,true,false> (attention + scatter epilogue)",
             "achieved": achieved,
             "peak": pk["bf16_sustained"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_sustained"],
             "traffic": ATTN_DRAM_BYTES_PER_KEPT_ROW * kept_rows,
