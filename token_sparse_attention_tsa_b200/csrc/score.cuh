@@ -32,7 +32,7 @@ namespace tsa {
 
 constexpr int SC_KEYS = 64;          // keys per tile (MMA N)
 constexpr int SC_ROWS = 128;         // window rows per block (MMA M)
-constexpr int SC_CHUNK_TILES = 16;   // key tiles per CTA (1024 keys)
+constexpr int SC_MIN_CHUNK_TILES = 16;   // smallest key span of a CTA, in tiles (1024 keys)
 constexpr int SC_THREADS = 192;
 constexpr int SC_STAGES = 3;
 
@@ -44,7 +44,8 @@ struct ScoreArgs {
   uint32_t* status;        // or null
   uint32_t* abort_word;    // launch-wide abort word (zeroed before launch) or null
   int L, w, Hq, Hkv, G;
-  int n_chunks;            // key chunks of SC_CHUNK_TILES tiles
+  int n_chunks;            // key chunks per head
+  int chunk_tiles;         // key tiles per chunk (one CTA each)
   int n_rb;                // window row blocks of 128
   float scale_log2;        // scale * log2(e)
   uint64_t limit_ns;
@@ -109,9 +110,9 @@ __global__ void __launch_bounds__(SC_THREADS, 1)
   const int Lb = a.seqs.len(b);                  // this sequence's length
   const int wb = a.w < Lb ? a.w : Lb;              // its window
   const int pos0 = Lb - wb;                        // position of window row 0
-  const int key0 = chunk * SC_CHUNK_TILES * SC_KEYS;
+  const int key0 = chunk * a.chunk_tiles * SC_KEYS;
   int n_kt = Lb > key0 ? (Lb - key0 + SC_KEYS - 1) / SC_KEYS : 0;
-  n_kt = n_kt > SC_CHUNK_TILES ? SC_CHUNK_TILES : n_kt;
+  n_kt = n_kt > a.chunk_tiles ? a.chunk_tiles : n_kt;
   const int steps = n_kt * a.n_rb;
   auto step_rb = [&](int s) { return kPass2 ? s % a.n_rb : s / n_kt; };
   auto step_kt = [&](int s) { return kPass2 ? s / a.n_rb : s % n_kt; };
@@ -325,7 +326,7 @@ static __global__ void score_merge_kernel(const ScoreArgs a, int total_rows) {
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= total_rows) return;
   const int Lb = a.seqs.len(idx / a.w / a.Hq);
-  constexpr int span = SC_CHUNK_TILES * SC_KEYS;
+  const int span = a.chunk_tiles * SC_KEYS;
   const int nc = (Lb + span - 1) / span;
   const float* pm = a.part_m + static_cast<size_t>(idx) * a.n_chunks;
   const double* pz = a.part_z + static_cast<size_t>(idx) * a.n_chunks;

@@ -31,8 +31,19 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// Key tiles per score CTA: long enough spans that the grid is a few waves of
+// 148 SMs (per-CTA set-up then amortises), never below 16 tiles.
+int score_chunk_tiles(const tsa_params* p) {
+  const int tiles = (p->L + tsa::SC_KEYS - 1) / tsa::SC_KEYS;
+  const int heads = p->B * p->Hq;
+  int per_head = (148 * 4) / heads;
+  per_head = per_head < 1 ? 1 : per_head;
+  const int ct = (tiles + per_head - 1) / per_head;
+  return ct < tsa::SC_MIN_CHUNK_TILES ? tsa::SC_MIN_CHUNK_TILES : ct;
+}
+
 int score_chunks(const tsa_params* p) {
-  const int span = tsa::SC_CHUNK_TILES * tsa::SC_KEYS;
+  const int span = score_chunk_tiles(p) * tsa::SC_KEYS;
   return (p->L + span - 1) / span;
 }
 
@@ -217,6 +228,7 @@ tsa_status run_score(const tsa_params* p, const void* q, const void* k, float* s
   a.Hkv = p->Hkv;
   a.G = p->Hq / p->Hkv;
   a.n_chunks = score_chunks(p);
+  a.chunk_tiles = score_chunk_tiles(p);
   a.n_rb = (p->w + tsa::SC_ROWS - 1) / tsa::SC_ROWS;
   a.scale_log2 = scale_of(p) * 1.4426950408889634f;
   a.limit_ns = limit_ns_of(p);
