@@ -71,3 +71,37 @@ def test_job_value_sums_ranks():
     assert abs(one - bench.dense_flops(wl) / 0.1 / 1e12) < 1e-9
     assert abs(bench.job_value(wl, 8, 100.0) - 8 * one) < 1e-6
     assert bench.max_over_ranks(3.5, None, None) == 3.5
+
+
+def test_compressed_flops_per_sequence_and_per_head():
+    """Attention FLOPs over kept rows: one count per sequence (every head
+    keeps it) equals the same count repeated per head."""
+    import numpy as np
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads as W
+    wl = W.WORKLOADS["c3_L32K_gqa_band"]
+    per_seq = np.array([25147])
+    per_head = np.full((1, wl.Hq), 25147)
+    a, b = bench.compressed_flops(wl, per_seq), bench.compressed_flops(wl, per_head)
+    assert a == b == wl.Hq * 2.0 * wl.d * 25147 * 25148
+    # heads keeping different counts
+    mixed = np.arange(1, wl.Hq + 1).reshape(1, wl.Hq) * 100
+    want = sum(2.0 * wl.d * n * (n + 1) for n in mixed.ravel())
+    assert bench.compressed_flops(wl, mixed) == want
+    # the full sequence kept gives the dense causal FLOPs
+    assert bench.compressed_flops(wl, np.array([wl.L])) == bench.dense_flops(wl)
+
+
+def test_both_arms_print_the_same_config():
+    import argparse
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads as W
+    wl = W.WORKLOADS["c4_L128K_gqa"]
+    args = argparse.Namespace(tau=0.05, budget_mode="max", keep_recent=0, layout="bhld", gpus=1)
+    cfg = bench.config_of(args, wl, 1)
+    assert cfg["workload"] == "c4_L128K_gqa" and cfg["L"] == 131072 and cfg["parallelism"] == "single"
+    assert bench.config_of(args, wl, 4)["parallelism"] == "replicas4"
