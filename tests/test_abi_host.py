@@ -139,6 +139,20 @@ def test_layer_switch_arguments(lib):
                  big, None) == INVALID                                          # dense branch: null v
 
 
+def test_block_mask_call_arguments(lib):
+    p = ctypes.byref(good())
+    ws_n = T.stage_workspace_size(good())
+    # qc, kc, vc, idx, k_seq, block_mask, o, lse, ws, ws_bytes, stream
+    assert _call(lib, "tsa_attend_blocks", p, FAKE, FAKE, FAKE, None, FAKE, None, FAKE, None, FAKE, ws_n,
+                 None) == INVALID                                            # no mask
+    assert _call(lib, "tsa_attend_blocks", p, FAKE, FAKE, FAKE, FAKE + 4, FAKE, FAKE, FAKE, None, FAKE, ws_n,
+                 None) == INVALID                                            # misaligned idx
+    assert _call(lib, "tsa_attend_blocks", p, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, None, FAKE, 8,
+                 None) == WORKSPACE                                          # workspace too small
+    assert _call(lib, "tsa_attend_blocks", None, FAKE, FAKE, FAKE, None, FAKE, FAKE, FAKE, None, FAKE, ws_n,
+                 None) == INVALID                                            # no params
+
+
 def test_per_head_budget_needs_head_counts(lib):
     p = ctypes.byref(good(budget_mode="per_head"))
     ws_n = T.stage_workspace_size(good(budget_mode="per_head"))
