@@ -80,7 +80,7 @@
 extern "C" {
 #endif
 
-#define TSA_ABI_VERSION 2
+#define TSA_ABI_VERSION 3
 
 typedef enum tsa_status {
   TSA_OK = 0,
@@ -99,6 +99,11 @@ typedef enum tsa_status {
  * TSA_DEVFLAG_TIMEOUT, lets its in-flight copies land, frees its tensor
  * memory and returns without writing outputs.  The context stays usable. */
 #define TSA_FLAG_TEST_STALL 0x80000000u
+/* The same test hook for the proxy-score kernels (tsa_score,
+ * tsa_score_noalloc, the score step of tsa_forward): the first score pass
+ * times out and sets TSA_DEVFLAG_TIMEOUT, every later score CTA of the call
+ * stops early, and the scores are not written. */
+#define TSA_FLAG_TEST_STALL_SCORE 0x40000000u
 
 /* tsa_params.budget_mode: how the heads' coverage counts k_head combine into
  * the rows each head keeps.  [GS] calls the budget global without saying how
@@ -123,7 +128,7 @@ typedef struct tsa_params {
   int32_t w;            /* proxy window: the last w query positions          */
   float tau;            /* coverage threshold, 0 <= tau < 1                  */
   float softmax_scale;  /* 0 selects 1/sqrt(d) (fp32)                        */
-  uint32_t flags;       /* 0, or TSA_FLAG_TEST_STALL (failure-path test)     */
+  uint32_t flags;       /* 0, or TSA_FLAG_TEST_STALL / _STALL_SCORE (tests)  */
   uint32_t timeout_ms;  /* limit of one pipeline wait; 0 selects 2000 ms     */
   int32_t budget_mode;  /* TSA_BUDGET_MAX (0), _MEAN or _PER_HEAD            */
   int32_t keep_recent;  /* 0 <= r <= L: the last r tokens of every sequence
@@ -145,8 +150,9 @@ const char* tsa_status_string(tsa_status s);
 tsa_status tsa_check_params(const tsa_params* p);
 
 /* Workspace bytes needed by tsa_forward (covers every stage call too): the
- * stage scratch, scores, indices, budgets and the compressed Q, K and V (no
- * compressed output is stored). */
+ * stage scratch, scores, indices, budgets and the compressed Q, K and V (the
+ * compressed output overwrites the compressed Q, so it takes no space of its
+ * own). */
 tsa_status tsa_workspace_size(const tsa_params* p, size_t* bytes);
 
 /* Workspace bytes needed by the single-stage calls below (status word and
@@ -214,8 +220,8 @@ tsa_status tsa_attend(const tsa_params* p, const void* qc, const void* kc, const
  * its epilogue.  [GS] "Arquitectura Central", decompression: compressed
  * output row i is written straight to o[b,h,S_h[i]] and every other row of o
  * is set to zero, so no compressed output is stored.  Same result as
- * tsa_attend followed by tsa_scatter; this is what tsa_forward runs after
- * tsa_gather_qkv.  In: qc, kc, vc (as tsa_attend), idx, k_seq.  Out: o
+ * tsa_attend followed by tsa_scatter.  In: qc, kc, vc (as tsa_attend), idx,
+ * k_seq.  Out: o
  * [B,Hq,L,d]; lse (nullable) indexed by compressed row.  An index outside
  * [0, L) is skipped and sets TSA_DEVFLAG_BAD_INDEX.  ws: stage size. */
 tsa_status tsa_attend_scatter(const tsa_params* p, const void* qc, const void* kc, const void* vc,
@@ -258,14 +264,18 @@ tsa_status tsa_attend_dense(const tsa_params* p, const void* q, const void* k, c
                             void* o, float* lse, void* ws, size_t ws_bytes, void* stream);
 
 /* Step 6 -- scatter.  [GS] "Arquitectura Central", decompression: o[b,h,:]
- * is zero except o[b,h,S_h[i]] = oc[b,h,i] for i < k_b.  Every row of o is
- * written exactly once.  ws: NULL or stage size. */
+ * is zero except o[b,h,S_h[i]] = oc[b,h,i] for i < k_b.  idx[b,h,0..k_b)
+ * must be strictly ascending, as tsa_select writes it: each CTA locates its
+ * rows by binary search.  With such an idx every row of o is written exactly
+ * once.  An entry outside [0, L_b) is not written and sets
+ * TSA_DEVFLAG_BAD_INDEX (when ws is not NULL).  ws: NULL or stage size. */
 tsa_status tsa_scatter(const tsa_params* p, const void* oc, const int32_t* idx, const int32_t* k_seq,
                        void* o, void* ws, size_t ws_bytes, void* stream);
 
-/* The whole path: score -> budget -> select -> gather -> attention writing
- * each output row in place, then zeros for the unselected rows (as
- * tsa_attend_scatter); enqueued on stream with no host synchronisation.
+/* The whole path: score -> budget -> select -> gather -> attention on the
+ * compressed tensors (its output written over the compressed Q in the
+ * workspace) -> scatter into o; enqueued on stream with no host
+ * synchronisation.
  * scores_out, idx_out, k_seq_out may be NULL (then the workspace holds
  * them); when given they receive the intermediate results, k_seq_out the
  * kept counts in the mode's shape ([B], or [B, Hq] in PER_HEAD mode).
@@ -273,6 +283,40 @@ tsa_status tsa_scatter(const tsa_params* p, const void* oc, const int32_t* idx, 
 tsa_status tsa_forward(const tsa_params* p, const void* q, const void* k, const void* v, void* o,
                        float* scores_out, int32_t* idx_out, int32_t* k_seq_out,
                        void* ws, size_t ws_bytes, void* stream);
+
+/* Head-sharded forward.  [GS] "Cobertura Dinamica de Tokens" makes the
+ * budget global across the heads of a sequence; every other step is per
+ * head.  When the query heads of one sequence are split over several devices
+ * (each holding whole heads: its query heads and the key/value heads they
+ * read), the forward runs in two halves around one exchange of B integers:
+ *
+ *   tsa_forward_begin   steps 1-2 on this device's heads: proxy scores and
+ *                       the per-head coverage counts k_head, plus this
+ *                       device's budget partial k_part [B]: the max of its
+ *                       k_head (TSA_BUDGET_MAX, and TSA_BUDGET_PER_HEAD where
+ *                       it is not used) or their sum (TSA_BUDGET_MEAN);
+ *   (the caller)        reduces k_part over the devices of the sequence's
+ *                       heads: MAX in MAX mode, SUM in MEAN mode, nothing in
+ *                       PER_HEAD mode (e.g. ncclAllReduce on B int32);
+ *   tsa_forward_end     the budget from the reduced value k_reduced (MAX: the
+ *                       value itself; MEAN: ceil(k_reduced / Hq_total);
+ *                       PER_HEAD: each head's own k_head), then steps 3-6.
+ *
+ * p describes this device's part (Hq, Hkv: its own head counts; every other
+ * field as for the whole problem); q, k, v, o are its heads' tensors.
+ * Hq_total is the number of query heads of a sequence over all devices
+ * (p->Hq when nothing is split).  On one device, begin + end with k_reduced =
+ * k_part compute exactly what tsa_forward computes.  Both halves take the
+ * same ws (>= tsa_workspace_size), which must not be touched in between;
+ * scores_out / scores and k_head_out / k_head may be NULL (the workspace
+ * then holds them) and, when given, must be the same buffers in both calls.
+ * k_part and k_reduced are DEVICE int32 [B] (k_reduced may be NULL in
+ * PER_HEAD mode); idx_out and k_seq_out are as in tsa_forward. */
+tsa_status tsa_forward_begin(const tsa_params* p, const void* q, const void* k, float* scores_out,
+                             int32_t* k_head_out, int32_t* k_part, void* ws, size_t ws_bytes, void* stream);
+tsa_status tsa_forward_end(const tsa_params* p, int32_t Hq_total, const void* q, const void* k, const void* v,
+                           void* o, const float* scores, const int32_t* k_head, const int32_t* k_reduced,
+                           int32_t* idx_out, int32_t* k_seq_out, void* ws, size_t ws_bytes, void* stream);
 
 /* Layer-level switch.  [GS] section 2 "Seleccion de Capas Dispersas" applies
  * the method only in the layers chosen by a criterion on the model's hidden
@@ -303,10 +347,20 @@ tsa_status tsa_layer_forward(const tsa_params* p, int32_t layer, const uint8_t* 
  * capture.  All calls share the one array and it keeps the last call's
  * contents: calls whose kernels overlap on the GPU (different streams, or
  * different host threads on one device) race and must be serialised by the
- * caller.  Calls no cudaMalloc, cudaFree or allocating library routine. */
+ * caller.  Calls no cudaMalloc, cudaFree or allocating library routine.
+ * Each call first clears the array's status word (enqueued on stream), so
+ * after it the word describes that call alone: a bounded pipeline wait that
+ * ran out (TSA_DEVFLAG_TIMEOUT, scores not written) or a sequence that did not
+ * fit.  Read it with tsa_score_noalloc_status. */
 #define TSA_NOALLOC_SCRATCH_BYTES (16u << 20)
 tsa_status tsa_score_noalloc(const tsa_params* p, const void* q, const void* k, float* scores,
                              void* stream);
+
+/* Status word of the most recent tsa_score_noalloc call on the current
+ * device, read without a workspace: synchronises stream, writes the raw bits
+ * to *flags (may be NULL) and maps them as tsa_get_device_status does.  No
+ * counterpart on the pages; allocates nothing. */
+tsa_status tsa_score_noalloc_status(void* stream, uint32_t* flags);
 
 #ifdef __cplusplus
 }

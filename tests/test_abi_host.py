@@ -42,7 +42,7 @@ def test_exports_every_declared_symbol(lib):
     assert len(names) == len(T.EXPORTED) and set(names) == set(T.EXPORTED)
     for n in names:
         assert hasattr(lib, n), n
-    assert lib.tsa_abi_version() == 2
+    assert lib.tsa_abi_version() == 3
 
 
 def test_status_strings(lib):
@@ -79,6 +79,10 @@ def test_flags_only_the_test_hook(lib):
     assert T.check_params(p) == INVALID
     p.flags = T.FLAG_TEST_STALL
     assert T.check_params(p) == 0
+    p.flags = T.FLAG_TEST_STALL_SCORE | T.FLAG_TEST_STALL
+    assert T.check_params(p) == 0
+    p.flags = T.FLAG_TEST_STALL_SCORE | 0x20000000
+    assert T.check_params(p) == INVALID
 
 
 def test_workspace_sizes(lib):

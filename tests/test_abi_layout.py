@@ -18,7 +18,8 @@ def c_layout():
     fields = [f for f, _ in T.tsa_params._fields_]
     body = "\n".join(f'  printf("{f} %zu\\n", offsetof(tsa_params, {f}));' for f in fields)
     src = ("#include <stddef.h>\n#include <stdio.h>\n#include \"tsa.h\"\n"
-           "int main(void) {\n" + body + '\n  printf("sizeof %zu\\n", sizeof(tsa_params));\n  return 0;\n}\n')
+           "int main(void) {\n" + body + '\n  printf("sizeof %zu\\n", sizeof(tsa_params));\n'
+           '  printf("noalloc_bytes %llu\\n", (unsigned long long)TSA_NOALLOC_SCRATCH_BYTES);\n  return 0;\n}\n')
     with tempfile.TemporaryDirectory() as d:
         c = os.path.join(d, "layout.c")
         exe = os.path.join(d, "layout")
@@ -36,6 +37,7 @@ def c_layout():
 def test_params_struct_layout_matches_the_header():
     lay = c_layout()
     assert lay.pop("sizeof") == ctypes.sizeof(T.tsa_params)
+    lay.pop("noalloc_bytes")
     for name, _ in T.tsa_params._fields_:
         assert lay[name] == getattr(T.tsa_params, name).offset, name
 
@@ -54,3 +56,8 @@ def test_params_struct_covers_every_header_field():
         names = decl.split(None, 1)[1] if not decl.startswith("const") else decl.split(None, 2)[2]
         declared += [n.strip().lstrip("*") for n in names.split(",")]
     assert declared == [f for f, _ in T.tsa_params._fields_]
+
+
+def test_noalloc_scratch_size_matches_the_header():
+    """The binding's copy of TSA_NOALLOC_SCRATCH_BYTES is the header's value."""
+    assert c_layout()["noalloc_bytes"] == T.NOALLOC_SCRATCH_BYTES

@@ -61,3 +61,29 @@ def test_forward_reports_timeout_then_recovers():
     qc, kc, vc = O.gather_qkv(q, k, v, g_idx, g_ks)
     ref = O.scatter(O.compressed_attention(qc, kc, vc, g_ks), g_idx, g_ks, WL.L)
     assert np.abs(bf16_to_f64(out) - ref).max() <= 2e-2
+
+
+def test_score_wait_runs_out_and_context_survives():
+    """TSA_FLAG_TEST_STALL_SCORE: the proxy-score kernel's bounded wait runs
+    out; the stage call and the forward report TIMEOUT (whatever else the
+    later steps flag on the unwritten scores), and normal calls that follow
+    on the same context are correct."""
+    (q, k, v), (dq, dk, dv) = inputs(WL)
+    stall = _params(timeout_ms=50, flags=T.FLAG_TEST_STALL_SCORE)
+    ws = T.new_workspace(stall, full=True)
+    scores = torch.full((WL.B, WL.Hq, WL.L), -3.0, device="cuda")
+    T.tsa_score(stall, dq, dk, scores, ws)
+    st, flags = T.get_device_status(ws)
+    assert st == TIMEOUT and flags & T.DEVFLAG_TIMEOUT
+    assert (scores == -3.0).all().item()          # not written
+    T.reset_device_status(ws)
+    o = torch.empty_like(dq)
+    T.tsa_forward(stall, dq, dk, dv, o, ws)
+    st, flags = T.get_device_status(ws)
+    assert st == TIMEOUT and flags & T.DEVFLAG_TIMEOUT
+    T.reset_device_status(ws)
+    T.tsa_score(_params(), dq, dk, scores, ws)
+    assert T.get_device_status(ws) == (0, 0)
+    _, s64 = O.proxy_scores(q, k, WL.w, return_f64=True)
+    err = np.abs(scores.cpu().numpy().astype(np.float64) - s64)
+    assert (err <= 1e-5 * np.abs(s64) + 1e-30).all()

@@ -3,10 +3,14 @@
 It exists for callers that cannot call cudaMalloc (a plug-in whose framework
 owns every device allocation, code under a hard memory budget, a C caller
 without an allocator): it takes no workspace and keeps its scratch in a fixed
-array inside the library.  Its output must match tsa_score, which takes the
-same scratch from a caller workspace, on two calls in a row (the array keeps
-the previous call's contents, so the second call checks that nothing stale is
-read).  This file is collected last so a failure here never hides the others.
+array inside the library.  It runs the same kernels as tsa_score on the same
+inputs, so its output must equal tsa_score's bit for bit, and both must lie
+within the score tolerance (1e-5 relative, element by element) of the fp64
+oracle -- on two calls in a row with a different call in between (the array
+keeps the previous call's contents, so this also checks that nothing stale is
+read).  Its status word is read through tsa_score_noalloc_status, which needs
+no workspace either.  This file is collected last so a failure here never
+hides the others.
 """
 import ctypes
 
@@ -14,35 +18,58 @@ import numpy as np
 import pytest
 import torch
 
+import oracle as O
 import token_sparse_attention_tsa_b200 as T
 import workloads as W
+from _gpu_util import scores_close
 
 pytestmark = pytest.mark.gpu
 
-SCORE_RTOL = 1e-5   # the score tolerance used by the parity tests
+TIMEOUT = 6
 
 
 def _dev(x):
     return torch.from_numpy(np.ascontiguousarray(x)).view(torch.bfloat16).cuda()
 
 
-def test_noalloc_scores_match_workspace_scores_twice():
+def _case(wl):
+    q, k, _ = W.generate(wl)
+    return q, k, _dev(q), _dev(k), T.params(wl.B, wl.Hq, wl.Hkv, wl.L, wl.d, wl.w, wl.tau)
+
+
+def test_noalloc_scores_equal_workspace_scores_twice():
     wl = W.WORKLOADS["c1_L1K_mha_d64"].with_(Hq=8, Hkv=2, L=3000, d=128, w=100, heavy_count=20, seed=21)
     wl2 = wl.with_(L=1500, w=64, seed=22)   # a different, smaller call in between
     outs = []
     for case in (wl, wl2, wl):
-        q, k, _ = (_dev(x) for x in W.generate(case))
-        p = T.params(case.B, case.Hq, case.Hkv, case.L, case.d, case.w, case.tau)
+        q, k, dq, dk, p = _case(case)
         ws = T.new_workspace(p, full=False)
         ref = torch.empty((case.B, case.Hq, case.L), device="cuda")
-        T.tsa_score(p, q, k, ref, ws)
+        T.tsa_score(p, dq, dk, ref, ws)
         got = torch.full_like(ref, float("nan"))
-        T.tsa_score_noalloc(p, q, k, got)
-        torch.cuda.synchronize()
-        r, g = ref.cpu().numpy().astype(np.float64), got.cpu().numpy().astype(np.float64)
-        assert np.all(np.abs(g - r) <= SCORE_RTOL * np.abs(r) + 1e-30)
-        outs.append(g)
-    assert np.array_equal(outs[0], outs[2])   # same input, same output after another call
+        T.tsa_score_noalloc(p, dq, dk, got)
+        assert T.score_noalloc_status() == (0, 0)
+        assert torch.equal(got.view(torch.int32), ref.view(torch.int32))       # same kernels: bit for bit
+        _, s64 = O.proxy_scores(q, k, case.w, return_f64=True)
+        assert scores_close(got.cpu().numpy(), s64) <= 1.0                     # 1e-5 relative
+        outs.append(got.cpu().numpy())
+    assert np.array_equal(outs[0].view(np.uint32), outs[2].view(np.uint32))   # same input, same output
+
+
+def test_noalloc_reports_a_timeout_and_the_next_call_is_clean():
+    wl = W.WORKLOADS["c1_L1K_mha_d64"].with_(Hq=4, Hkv=2, L=2000, d=128, w=64, seed=23)
+    q, k, dq, dk, p = _case(wl)
+    stall = T.params(wl.B, wl.Hq, wl.Hkv, wl.L, wl.d, wl.w, wl.tau, timeout_ms=50, flags=T.FLAG_TEST_STALL_SCORE)
+    got = torch.full((wl.B, wl.Hq, wl.L), -3.0, device="cuda")
+    T.tsa_score_noalloc(stall, dq, dk, got)
+    st, flags = T.score_noalloc_status()
+    assert st == TIMEOUT and flags & T.DEVFLAG_TIMEOUT
+    assert (got == -3.0).all().item()          # the scores were not written
+    # the next call clears the status word and is correct
+    T.tsa_score_noalloc(p, dq, dk, got)
+    assert T.score_noalloc_status() == (0, 0)
+    _, s64 = O.proxy_scores(q, k, wl.w, return_f64=True)
+    assert scores_close(got.cpu().numpy(), s64) <= 1.0
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():

@@ -24,6 +24,7 @@ STATUS_NAMES = {0: "TSA_OK", 1: "TSA_ERR_INVALID_ARG", 2: "TSA_ERR_UNSUPPORTED",
                 4: "TSA_ERR_CUDA", 5: "TSA_ERR_NONFINITE", 6: "TSA_ERR_TIMEOUT", 7: "TSA_ERR_BAD_INDEX"}
 DEVFLAG_NONFINITE, DEVFLAG_TIMEOUT, DEVFLAG_BAD_INDEX = 0x1, 0x2, 0x4
 FLAG_TEST_STALL = 0x80000000
+FLAG_TEST_STALL_SCORE = 0x40000000
 BUDGET_MAX, BUDGET_MEAN, BUDGET_PER_HEAD = 0, 1, 2
 BUDGET_MODES = {"max": BUDGET_MAX, "mean": BUDGET_MEAN, "per_head": BUDGET_PER_HEAD}
 LAYOUT_BHLD, LAYOUT_BLHD = 0, 1
@@ -34,7 +35,8 @@ EXPORTED = ("tsa_abi_version", "tsa_status_string", "tsa_check_params", "tsa_wor
             "tsa_stage_workspace_size", "tsa_reset_device_status", "tsa_get_device_status",
             "tsa_score", "tsa_budget", "tsa_select", "tsa_gather_qkv", "tsa_attend",
             "tsa_attend_dense", "tsa_attend_scatter", "tsa_attend_gathered", "tsa_attend_blocks", "tsa_scatter",
-            "tsa_forward", "tsa_layer_forward", "tsa_score_noalloc")
+            "tsa_forward", "tsa_forward_begin", "tsa_forward_end", "tsa_layer_forward", "tsa_score_noalloc",
+            "tsa_score_noalloc_status")
 
 
 class TSAError(RuntimeError):
@@ -113,9 +115,13 @@ def load(path: str | None = None):
             "tsa_attend_blocks": ([_P, _v, _v, _v, _v, _v, _v, _v, _v, _v, _sz, _v], ctypes.c_int),
             "tsa_scatter": ([_P, _v, _v, _v, _v, _v, _sz, _v], ctypes.c_int),
             "tsa_forward": ([_P, _v, _v, _v, _v, _v, _v, _v, _v, _sz, _v], ctypes.c_int),
+            "tsa_forward_begin": ([_P, _v, _v, _v, _v, _v, _v, _sz, _v], ctypes.c_int),
+            "tsa_forward_end": ([_P, ctypes.c_int32, _v, _v, _v, _v, _v, _v, _v, _v, _v, _v, _sz, _v],
+                                ctypes.c_int),
             "tsa_layer_forward": ([_P, ctypes.c_int32, _v, ctypes.c_int32, _v, _v, _v, _v, _v, _v, _v, _v, _sz, _v],
                                   ctypes.c_int),
             "tsa_score_noalloc": ([_P, _v, _v, _v, _v], ctypes.c_int),
+            "tsa_score_noalloc_status": ([_v, ctypes.POINTER(ctypes.c_uint32)], ctypes.c_int),
         }
         for name, (args, res) in sig.items():
             fn = getattr(lib, name)
@@ -210,7 +216,7 @@ def tsa_score(p, q, k, scores, ws, stream=None):
                             _stream(stream)), "tsa_score")
 
 
-NOALLOC_SCRATCH_BYTES = 16 << 20
+NOALLOC_SCRATCH_BYTES = 16 << 20   # TSA_NOALLOC_SCRATCH_BYTES of the header
 
 
 def tsa_score_noalloc(p, q, k, scores, stream=None):
@@ -220,6 +226,14 @@ def tsa_score_noalloc(p, q, k, scores, stream=None):
     import torch
     _check(load().tsa_score_noalloc(ctypes.byref(p), _ptr(q, "q", torch.bfloat16), _ptr(k, "k", torch.bfloat16),
                                     _ptr(scores, "scores", torch.float32), _stream(stream)), "tsa_score_noalloc")
+
+
+def score_noalloc_status(stream=None) -> tuple[int, int]:
+    """(status code, raw flag bits) of the most recent tsa_score_noalloc call
+    on the current device; synchronises."""
+    flags = ctypes.c_uint32()
+    st = load().tsa_score_noalloc_status(_stream(stream), ctypes.byref(flags))
+    return st, flags.value
 
 
 def tsa_budget(p, scores, k_head, k_seq, ws, stream=None):
@@ -307,6 +321,72 @@ def tsa_forward(p, q, k, v, o, ws, scores_out=None, idx_out=None, k_seq_out=None
                               _ptr(o, "o", bf), _ptr(scores_out, "scores_out", torch.float32),
                               _ptr(idx_out, "idx_out", torch.int32), _ptr(k_seq_out, "k_seq_out", torch.int32),
                               _ptr(ws, "ws"), _nbytes(ws), _stream(stream)), "tsa_forward")
+
+
+def tsa_forward_begin(p, q, k, k_part, ws, scores_out=None, k_head_out=None, stream=None):
+    import torch
+    bf = torch.bfloat16
+    _check(load().tsa_forward_begin(ctypes.byref(p), _ptr(q, "q", bf), _ptr(k, "k", bf),
+                                    _ptr(scores_out, "scores_out", torch.float32),
+                                    _ptr(k_head_out, "k_head_out", torch.int32), _ptr(k_part, "k_part", torch.int32),
+                                    _ptr(ws, "ws"), _nbytes(ws), _stream(stream)), "tsa_forward_begin")
+
+
+def tsa_forward_end(p, Hq_total: int, q, k, v, o, k_reduced, ws, scores=None, k_head=None, idx_out=None,
+                    k_seq_out=None, stream=None):
+    import torch
+    bf = torch.bfloat16
+    _check(load().tsa_forward_end(ctypes.byref(p), int(Hq_total), _ptr(q, "q", bf), _ptr(k, "k", bf),
+                                  _ptr(v, "v", bf), _ptr(o, "o", bf), _ptr(scores, "scores", torch.float32),
+                                  _ptr(k_head, "k_head", torch.int32), _ptr(k_reduced, "k_reduced", torch.int32),
+                                  _ptr(idx_out, "idx_out", torch.int32), _ptr(k_seq_out, "k_seq_out", torch.int32),
+                                  _ptr(ws, "ws"), _nbytes(ws), _stream(stream)), "tsa_forward_end")
+
+
+# ---------------------------------------------------------------- head sharding
+def budget_reduce_op(budget_mode) -> str | None:
+    """How the budget partials of tsa_forward_begin combine over the devices
+    that share a sequence's heads: "max" (MAX mode), "sum" (MEAN mode: the
+    partials are count sums) or None (PER_HEAD mode: nothing is shared)."""
+    if isinstance(budget_mode, str):
+        budget_mode = BUDGET_MODES[budget_mode]
+    return {BUDGET_MAX: "max", BUDGET_MEAN: "sum", BUDGET_PER_HEAD: None}[budget_mode]
+
+
+def shard_heads(Hq: int, Hkv: int, world: int, rank: int) -> tuple[int, int, int, int]:
+    """Heads of `rank` when a sequence's Hq query heads are split evenly over
+    `world` devices: query heads [h0, h1) and the key/value heads [kv0, kv1)
+    they read (query head h reads KV head h // (Hq // Hkv)).  Each device
+    holds whole GQA groups, or a whole divisor of one group (its KV head is
+    then also held by the other devices of that group)."""
+    if world < 1 or not 0 <= rank < world:
+        raise ValueError(f"rank {rank} of {world}")
+    if Hq % Hkv or Hq % world:
+        raise ValueError(f"Hq={Hq} must be divisible by Hkv={Hkv} and by world={world}")
+    G = Hq // Hkv
+    n = Hq // world
+    if n % G and G % n:
+        raise ValueError(f"{n} query heads per device split a group of {G} unevenly")
+    h0, h1 = rank * n, (rank + 1) * n
+    return h0, h1, h0 // G, (h1 - 1) // G + 1
+
+
+def forward_sharded(p, Hq_total: int, q, k, v, o, ws, group=None, scores_out=None, idx_out=None, k_seq_out=None):
+    """The forward of this device's heads of a head-sharded batch (p, q, k, v,
+    o describe the local heads; Hq_total counts a sequence's query heads over
+    all devices): tsa_forward_begin, one all-reduce of the B budget partials
+    over `group` (torch.distributed, e.g. NCCL; skipped when nothing is
+    shared or the group has one member), tsa_forward_end.  Runs on the
+    current CUDA stream."""
+    import torch
+    import torch.distributed as dist
+    k_part = torch.empty((p.B,), dtype=torch.int32, device=q.device)
+    tsa_forward_begin(p, q, k, k_part, ws, scores_out=scores_out)
+    op = budget_reduce_op(p.budget_mode)
+    if op is not None and dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:
+        dist.all_reduce(k_part, op=dist.ReduceOp.MAX if op == "max" else dist.ReduceOp.SUM, group=group)
+    tsa_forward_end(p, Hq_total, q, k, v, o, k_part, ws, scores=scores_out, idx_out=idx_out, k_seq_out=k_seq_out)
+    return k_part
 
 
 def tsa_layer_forward(p, layer: int, sparse_layers, q, k, v, o, ws, scores_out=None, idx_out=None, k_seq_out=None,

@@ -107,11 +107,14 @@ __global__ void __launch_bounds__(256) scatter_kernel(const ScatterArgs a) {
   __syncthreads();
   bool bad = false;
   {
+    // an entry outside [0, L_b), or one not above its predecessor (idx must
+    // ascend strictly for the binary search above), is reported, not written
     const int i = s_first + threadIdx.x;
     if (i < kb) {
-      const int r = __ldg(ix + i) - r0;
-      if (r >= 0 && r < SCAT_ROWS) where[r] = i;
-      else if (r + r0 < 0 || r + r0 >= Lb) bad = true;
+      const int j = __ldg(ix + i);
+      const int r = j - r0;
+      if (j < 0 || j >= Lb || (i > 0 && __ldg(ix + i - 1) >= j)) bad = true;
+      else if (r >= 0 && r < SCAT_ROWS) where[r] = i;
     }
   }
   __syncthreads();

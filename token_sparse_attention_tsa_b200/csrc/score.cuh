@@ -50,6 +50,7 @@ struct ScoreArgs {
   float scale_log2;        // scale * log2(e)
   uint64_t limit_ns;
   int token_major;         // q, k maps are (d, H, L, B) (else (d, L, H, B))
+  int test_stall;          // failure-path test: the MMA issuer first waits on a barrier nothing completes
   Seqs seqs;               // sequence lengths (and packed token offsets)
 };
 
@@ -176,7 +177,10 @@ __global__ void __launch_bounds__(SC_THREADS, 1)
     // ------------------------------------------------------------ MMA issuer
     const bool leader = elect_one();
     constexpr uint32_t idS = idesc_bf16_f32(128, SC_KEYS, 0, 0);
-    for (int s = 0; s < steps; ++s) {
+    // test hook: phase 0 of the drain barrier completes only at teardown, so
+    // this bounded wait runs out and the CTA takes the abort path
+    const bool stalled = a.test_stall && !__all_sync(0xffffffffu, mbar_wait(bar(SB_DRAIN), 0, wc));
+    for (int s = 0; !stalled && s < steps; ++s) {
       const int st = s % SC_STAGES, buf = s & 1;
       if (!__all_sync(0xffffffffu, mbar_wait(bar(SB_FULL + st), (s / SC_STAGES) & 1, wc))) break;
       if (s >= 2 && !__all_sync(0xffffffffu, mbar_wait(bar(SB_SFREE + buf), ((s >> 1) - 1) & 1, wc))) break;

@@ -204,8 +204,10 @@ __global__ void __launch_bounds__(BS_THREADS, 1) budget_kernel(const BudgetArgs 
   if (a.status && __syncthreads_or(bad) && threadIdx.x == 0) atomicOr(a.status, 0x1u);
 }
 
-// k_seq[b] from the heads' counts: mode 1 the ceiling of their mean, else
-// their maximum.  grid: B CTAs of 32 threads.
+// k_seq[b] from the heads' counts: mode 1 the ceiling of their mean, mode 2
+// their sum (the partial a device contributes when a sequence's heads are
+// split over devices and the budget is the mean), else their maximum.
+// grid: B CTAs of 32 threads.
 __global__ void __launch_bounds__(32) budget_finalize_kernel(const int32_t* k_head, int32_t* k_seq, int Hq,
                                                              int mode) {
   const int b = blockIdx.x;
@@ -222,7 +224,19 @@ __global__ void __launch_bounds__(32) budget_finalize_kernel(const int32_t* k_he
     const int y = __shfl_xor_sync(0xffffffffu, mx, o);
     mx = y > mx ? y : mx;
   }
-  if (threadIdx.x == 0) k_seq[b] = mode == 1 ? static_cast<int32_t>((sum + Hq - 1) / Hq) : mx;
+  if (threadIdx.x == 0)
+    k_seq[b] = mode == 1 ? static_cast<int32_t>((sum + Hq - 1) / Hq) : (mode == 2 ? static_cast<int32_t>(sum) : mx);
+}
+
+// The mean-mode budget from the heads' count sum over all devices:
+// k_seq[b] = ceil(k_sum[b] / Hq_total) (in place allowed).  One thread per
+// sequence.
+__global__ void __launch_bounds__(128) budget_mean_kernel(const int32_t* k_sum, int32_t* k_seq, int B,
+                                                          int Hq_total) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= B) return;
+  const long long s = k_sum[b];
+  k_seq[b] = static_cast<int32_t>((s + Hq_total - 1) / Hq_total);
 }
 
 struct SelectArgs {

@@ -237,10 +237,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
-}  // namespace tsa
-
-namespace tsa {
-
 // D[tmem] (+)= A[tmem] * B[smem desc]^T, kind::f16: A (M x K bf16) is read
 // from TMEM, row m in lane m, two K elements per 32-bit column.
 __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
@@ -252,11 +248,6 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       : "memory");
 }
 
-// Store 32 consecutive 32-bit columns of this thread's TMEM lane.
-}  // namespace tsa
-
-namespace tsa {
-
 // Store 16 consecutive 32-bit columns of this thread's TMEM lane.
 __device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t (&u)[16]) {
   asm volatile(
@@ -267,11 +258,6 @@ __device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t (&u)[1
       "r"(u[15])
       : "memory");
 }
-
-}  // namespace tsa
-
-
-namespace tsa {
 
 // Named barrier over `count` threads that also ANDs a predicate across them,
 // so every participant takes the same branch afterwards.
@@ -286,10 +272,6 @@ __device__ __forceinline__ bool bar_and(uint32_t id, uint32_t count, bool v) {
   return r != 0;
 }
 
-}  // namespace tsa
-
-namespace tsa {
-
 // One lane of the (fully active) warp is elected; every lane gets whether it
 // is the one.  Used so that loops around single-thread tcgen05/TMA issue run
 // warp-wide on uniform values.
@@ -302,10 +284,6 @@ __device__ __forceinline__ bool elect_one() {
   return pred != 0;
 }
 
-}  // namespace tsa
-
-namespace tsa {
-
 // TMA row gather: rows r0..r3 (x columns from col) of a 2D tensor map whose
 // box is one row high land as four consecutive rows at dst.
 __device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* m, uint32_t bar, int col, int r0,
@@ -316,10 +294,6 @@ __device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* m, 
       "l"(reinterpret_cast<uint64_t>(m)), "r"(bar), "r"(col), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
       : "memory");
 }
-
-}  // namespace tsa
-
-namespace tsa {
 
 // Packed fp32x2 arithmetic (two fp32 lanes in one 64-bit register): one
 // instruction does the work of two, which matters in the issue-bound softmax.

@@ -233,6 +233,7 @@ tsa_status run_score(const tsa_params* p, const void* q, const void* k, float* s
   a.scale_log2 = scale_of(p) * 1.4426950408889634f;
   a.limit_ns = limit_ns_of(p);
   a.token_major = tm ? 1 : 0;
+  a.test_stall = (p->flags & TSA_FLAG_TEST_STALL_SCORE) ? 1 : 0;
   a.seqs = seqs_of(p);
   const dim3 grid(a.n_chunks, bhq);
   const int rows = bhq * p->w;
@@ -259,15 +260,16 @@ tsa_status run_score(const tsa_params* p, const void* q, const void* k, float* s
 
 // k_head receives every head's count (required); k_seq, when not null, the
 // per-sequence budget of the mode (max, or ceiling of the mean; per-head
-// mode reports the max).
+// mode reports the max).  partial: k_seq receives this device's share of a
+// budget combined over devices instead (the sum of the counts in mean mode,
+// the max otherwise).
 tsa_status run_budget(const tsa_params* p, const float* scores, int32_t* k_head, int32_t* k_seq,
-                      uint32_t* status, cudaStream_t st) {
+                      uint32_t* status, cudaStream_t st, bool partial = false) {
   if (!ensure_smem(g_budget, tsa::budget_kernel, kBudgetSmem)) return TSA_ERR_CUDA;
   tsa::BudgetArgs a{scores, k_head, status, p->L, p->Hq, p->keep_recent, static_cast<double>(p->tau), seqs_of(p)};
   tsa::budget_kernel<<<p->B * p->Hq, tsa::BS_THREADS, kBudgetSmem, st>>>(a);
-  if (k_seq)
-    tsa::budget_finalize_kernel<<<p->B, 32, 0, st>>>(k_head, k_seq, p->Hq,
-                                                     p->budget_mode == TSA_BUDGET_MEAN ? 1 : 0);
+  const bool mean = p->budget_mode == TSA_BUDGET_MEAN;
+  if (k_seq) tsa::budget_finalize_kernel<<<p->B, 32, 0, st>>>(k_head, k_seq, p->Hq, mean ? (partial ? 2 : 1) : 0);
   return launch_ok();
 }
 
@@ -457,7 +459,7 @@ tsa_status tsa_check_params(const tsa_params* p) {
   if (p->w > p->L) return TSA_ERR_INVALID_ARG;
   if (!(p->tau >= 0.f && p->tau < 1.f)) return TSA_ERR_INVALID_ARG;
   if (!(p->softmax_scale >= 0.f) || std::isinf(p->softmax_scale)) return TSA_ERR_INVALID_ARG;
-  if ((p->flags & ~TSA_FLAG_TEST_STALL) != 0) return TSA_ERR_INVALID_ARG;
+  if ((p->flags & ~(TSA_FLAG_TEST_STALL | TSA_FLAG_TEST_STALL_SCORE)) != 0) return TSA_ERR_INVALID_ARG;
   if (p->budget_mode < TSA_BUDGET_MAX || p->budget_mode > TSA_BUDGET_PER_HEAD) return TSA_ERR_INVALID_ARG;
   if (p->keep_recent < 0 || p->keep_recent > p->L) return TSA_ERR_INVALID_ARG;
   if (p->layout != TSA_LAYOUT_BHLD && p->layout != TSA_LAYOUT_BLHD) return TSA_ERR_INVALID_ARG;
@@ -577,15 +579,48 @@ tsa_status tsa_scatter(const tsa_params* p, const void* oc, const int32_t* idx, 
   return run_scatter(p, oc, idx, k_seq, o, status_of(ws), static_cast<cudaStream_t>(stream));
 }
 
+}  // extern "C"
+
+namespace {
+
+// Steps 3-6 of the forward from the scores and the kept counts: selection,
+// gather, attention (output over qc in place) and scatter.
+tsa_status forward_tail(const tsa_params* p, const void* q, const void* k, const void* v, void* o,
+                        const float* scores, const int32_t* kseq, int32_t* idx, void* ws, cudaStream_t st) {
+  const WsLayout w = layout_of(p);
+  tsa_status s;
+  if ((s = run_select(p, scores, kseq, idx, st)) != TSA_OK) return s;
+  // gather once; attention on the compressed tensors with its output written
+  // over qc in place (each CTA loads its own two query tiles into shared
+  // memory before any of its output rows is stored, and no other CTA reads
+  // them); then the scatter writes every row of o once
+  // (tsa_gather_qkv + tsa_attend with oc = qc + tsa_scatter)
+  void* qc = at<void>(ws, w.qc);
+  void* kc = at<void>(ws, w.kc);
+  void* vc = at<void>(ws, w.vc);
+  if ((s = run_gather(p, q, k, v, idx, kseq, qc, kc, vc, status_of(ws), st)) != TSA_OK) return s;
+  if ((s = run_attend(p, qc, kc, vc, p->Hq, 1, kseq, qc, nullptr, status_of(ws), abort_of(ws), st, false,
+                      false)) != TSA_OK)
+    return s;
+  return run_scatter(p, qc, idx, kseq, o, status_of(ws), st);
+}
+
+bool out_ptrs_ok(const float* scores, const int32_t* idx, const int32_t* kvec, const int32_t* kseq) {
+  return !(scores && !aligned(scores, 16)) && !(idx && !aligned(idx, 16)) && !(kvec && !aligned(kvec, 4)) &&
+         !(kseq && !aligned(kseq, 4));
+}
+
+}  // namespace
+
+extern "C" {
+
 tsa_status tsa_forward(const tsa_params* p, const void* q, const void* k, const void* v, void* o,
                        float* scores_out, int32_t* idx_out, int32_t* k_seq_out, void* ws, size_t ws_bytes,
                        void* stream) {
   tsa_status s = tsa_check_params(p);
   if (s != TSA_OK) return s;
   if (!tensors_ok({q, k, v, o})) return TSA_ERR_INVALID_ARG;
-  if ((scores_out && !aligned(scores_out, 16)) || (idx_out && !aligned(idx_out, 16)) ||
-      (k_seq_out && !aligned(k_seq_out, 4)))
-    return TSA_ERR_INVALID_ARG;
+  if (!out_ptrs_ok(scores_out, idx_out, nullptr, k_seq_out)) return TSA_ERR_INVALID_ARG;
   if ((s = check_ws(p, ws, ws_bytes, true)) != TSA_OK) return s;
   const WsLayout w = layout_of(p);
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -597,17 +632,59 @@ tsa_status tsa_forward(const tsa_params* p, const void* q, const void* k, const 
   int32_t* kseq = per_head(p) ? khead : kbud;
   if ((s = run_score(p, q, k, scores, ws, st)) != TSA_OK) return s;
   if ((s = run_budget(p, scores, khead, kbud, status_of(ws), st)) != TSA_OK) return s;
-  if ((s = run_select(p, scores, kseq, idx, st)) != TSA_OK) return s;
-  // gather once, attention writing each output row in place, zeros for the
-  // unselected rows (tsa_gather_qkv + tsa_attend_scatter)
-  void* qc = at<void>(ws, w.qc);
-  void* kc = at<void>(ws, w.kc);
-  void* vc = at<void>(ws, w.vc);
-  if ((s = run_gather(p, q, k, v, idx, kseq, qc, kc, vc, status_of(ws), st)) != TSA_OK) return s;
-  if ((s = run_attend(p, qc, kc, vc, p->Hq, 1, kseq, o, nullptr, status_of(ws), abort_of(ws), st, false, true,
-                      idx)) != TSA_OK)
-    return s;
-  return run_zero_unselected(p, idx, kseq, o, status_of(ws), st);
+  return forward_tail(p, q, k, v, o, scores, kseq, idx, ws, st);
+}
+
+tsa_status tsa_forward_begin(const tsa_params* p, const void* q, const void* k, float* scores_out,
+                             int32_t* k_head_out, int32_t* k_part, void* ws, size_t ws_bytes, void* stream) {
+  tsa_status s = tsa_check_params(p);
+  if (s != TSA_OK) return s;
+  if (!tensors_ok({q, k}) || !k_part || !aligned(k_part, 4)) return TSA_ERR_INVALID_ARG;
+  if (!out_ptrs_ok(scores_out, nullptr, k_head_out, nullptr)) return TSA_ERR_INVALID_ARG;
+  if ((s = check_ws(p, ws, ws_bytes, true)) != TSA_OK) return s;
+  const WsLayout w = layout_of(p);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* scores = scores_out ? scores_out : at<float>(ws, w.scores);
+  int32_t* khead = k_head_out ? k_head_out : at<int32_t>(ws, w.k_head);
+  if ((s = run_score(p, q, k, scores, ws, st)) != TSA_OK) return s;
+  return run_budget(p, scores, khead, k_part, status_of(ws), st, true);
+}
+
+tsa_status tsa_forward_end(const tsa_params* p, int32_t Hq_total, const void* q, const void* k, const void* v,
+                           void* o, const float* scores, const int32_t* k_head, const int32_t* k_reduced,
+                           int32_t* idx_out, int32_t* k_seq_out, void* ws, size_t ws_bytes, void* stream) {
+  tsa_status s = tsa_check_params(p);
+  if (s != TSA_OK) return s;
+  if (Hq_total < p->Hq) return TSA_ERR_INVALID_ARG;
+  if (static_cast<long long>(p->B) * Hq_total * p->L >= (1LL << 31)) return TSA_ERR_UNSUPPORTED;
+  if (!tensors_ok({q, k, v, o})) return TSA_ERR_INVALID_ARG;
+  if (!per_head(p) && (!k_reduced || !aligned(k_reduced, 4))) return TSA_ERR_INVALID_ARG;
+  if (!out_ptrs_ok(scores, idx_out, k_head, k_seq_out)) return TSA_ERR_INVALID_ARG;
+  if ((s = check_ws(p, ws, ws_bytes, true)) != TSA_OK) return s;
+  const WsLayout w = layout_of(p);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const float* sc = scores ? scores : at<float>(ws, w.scores);
+  int32_t* idx = idx_out ? idx_out : at<int32_t>(ws, w.idx);
+  const int32_t* kseq = nullptr;
+  if (per_head(p)) {  // nothing is combined over heads: each head keeps its own count
+    const int32_t* kh = k_head ? k_head : at<int32_t>(ws, w.k_head);
+    if (k_seq_out && cudaMemcpyAsync(k_seq_out, kh, static_cast<size_t>(p->B) * p->Hq * sizeof(int32_t),
+                                     cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+      return TSA_ERR_CUDA;
+    kseq = kh;
+  } else if (p->budget_mode == TSA_BUDGET_MEAN) {  // the reduced value is the sum of every head's count
+    int32_t* kb = k_seq_out ? k_seq_out : at<int32_t>(ws, w.k_seq);
+    tsa::budget_mean_kernel<<<(p->B + 127) / 128, 128, 0, st>>>(k_reduced, kb, p->B, Hq_total);
+    if ((s = launch_ok()) != TSA_OK) return s;
+    kseq = kb;
+  } else {  // the reduced value is the max over every head's count: the budget itself
+    if (k_seq_out && k_seq_out != k_reduced &&
+        cudaMemcpyAsync(k_seq_out, k_reduced, static_cast<size_t>(p->B) * sizeof(int32_t),
+                        cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+      return TSA_ERR_CUDA;
+    kseq = k_reduced;
+  }
+  return forward_tail(p, q, k, v, o, sc, kseq, idx, ws, st);
 }
 
 tsa_status tsa_attend_scatter(const tsa_params* p, const void* qc, const void* kc, const void* vc,
@@ -710,7 +787,18 @@ extern "C" tsa_status tsa_score_noalloc(const tsa_params* p, const void* q, cons
   if (layout_of(p).stage_end > static_cast<size_t>(TSA_NOALLOC_SCRATCH_BYTES)) return TSA_ERR_WORKSPACE;
   void* scratch = nullptr;
   if ((s = scratch_address(&scratch)) != TSA_OK) return s;
-  // Every scratch entry the kernels read is written earlier in the same call,
-  // so nothing has to be cleared between calls.
-  return run_score(p, q, k, scores, scratch, static_cast<cudaStream_t>(stream));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // The status and abort words at the start of the array describe this call
+  // only: clear them first.  Every other scratch entry the kernels read is
+  // written earlier in the same call when no CTA aborts; after an abort the
+  // status word says so and the scores are not to be used.
+  if (cudaMemsetAsync(scratch, 0, 16, st) != cudaSuccess) return TSA_ERR_CUDA;
+  return run_score(p, q, k, scores, scratch, st);
+}
+
+extern "C" tsa_status tsa_score_noalloc_status(void* stream, uint32_t* flags) {
+  void* scratch = nullptr;
+  const tsa_status s = scratch_address(&scratch);
+  if (s != TSA_OK) return s;
+  return tsa_get_device_status(scratch, stream, flags);
 }
