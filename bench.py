@@ -9,8 +9,11 @@ kernel on the same tensors is reported beside it).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--tau T] [--impl reference]
 
-With --gpus N > 1 (under torchrun) every rank runs its own sequence: the
-units shard across ranks with no data-path collective (weak scaling); the
+With --gpus N > 1 (under torchrun) the ranks split the query heads of the
+one sequence (--shard heads, the default: every step runs on each rank's
+heads, and the budget, which is global over a sequence's heads, is combined
+by one all-reduce of B integers per step; strong scaling), or every rank
+runs its own sequence (--shard replicas: no collective; weak scaling).  The
 step time is the max over ranks.  --impl reference times the CPU oracle on a
 bounded sample of the same workload on the host cores (rank 0 only).
 """
@@ -36,12 +39,42 @@ import workloads as W  # noqa: E402
 METRIC = "Token-sparse prefill attention ms and effective TFLOP/s at 128K vs dense; % BF16/HBM roofline"
 UNIT = "TFLOP/s (effective: dense causal attention FLOPs / TSA time)"
 DEFAULT_WORKLOAD = "c4_L128K_gqa"
-KERNELS_PER_FORWARD = 9  # score x3, budget, budget finalize, select, gather, attention (scatter epilogue), zero fill
-# DRAM bytes per kept (head, row) of the attention kernel with the scatter
-# epilogue, from ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch
-# on the 32K workload (811.5 MB for 32 x 25147 kept rows); DRAM traffic grows
-# with kept rows, not with FLOPs (algorithmic: 3 x 256 B read + 256 B written).
-ATTN_DRAM_BYTES_PER_KEPT_ROW = 811.5e6 / (32 * 25147)
+KERNELS_PER_FORWARD = 9  # score x3, budget, budget finalize, select, gather, attention, scatter
+# DRAM bytes per kept (head, row) of the forward's attention kernel, from ncu
+# dram__bytes_read.sum + dram__bytes_write.sum of one launch (None until the
+# current kernel has been captured); DRAM traffic grows with kept rows, not
+# with FLOPs (algorithmic: 3 x 256 B read + 256 B written per kept row).
+ATTN_DRAM_BYTES_PER_KEPT_ROW = None
+ATTN_TRAFFIC_NOTE = "not yet captured for the current kernel"
+SMS = 148
+EX2_PER_CLK_SM = 32
+
+
+def stage_algorithmic_bytes(wl, kept_np, idx) -> dict:
+    """Algorithmic HBM bytes of the HBM-bound stages for one forward.
+
+    gather:  Q rows of every kept (head, row), the UNIQUE K and V rows each
+             KV group reads (the union of its query heads' selections), and
+             the three compressed rows written per kept (head, row);
+    scatter: every output row written plus the kept compressed rows read;
+    score:   one read of K, the window rows of Q, and the fp32 scores.
+    idx: the device index tensor [B, Hq, L] of the forward just timed."""
+    import torch
+    B, Hq, Hkv, L, d = wl.B, wl.Hq, wl.Hkv, wl.L, wl.d
+    G = Hq // Hkv
+    per_head = kept_np if kept_np.ndim == 2 else np.repeat(np.asarray(kept_np)[:, None], Hq, axis=1)
+    kept = int(per_head.sum())
+    row = d * 2
+    uniq = 0
+    for b in range(B):
+        for g in range(Hkv):
+            mask = torch.zeros(L, dtype=torch.bool, device=idx.device)
+            for h in range(g * G, (g + 1) * G):
+                mask[idx[b, h, :int(per_head[b, h])].long()] = True
+            uniq += int(mask.sum().item())
+    return {"gather": kept * row + 2 * uniq * row + 3 * kept * row,
+            "scatter": B * Hq * L * row + kept * row,
+            "score": B * Hkv * L * row + B * Hq * wl.w * row + B * Hq * L * 4}
 
 
 def dense_flops(wl) -> float:
@@ -82,10 +115,11 @@ def max_over_ranks(x: float, dist, device) -> float:
     return float(t.item())
 
 
-def job_value(wl, world: int, ms: float) -> float:
-    """Whole-job effective TFLOP/s: every rank's dense-equivalent FLOPs over
-    the max-over-ranks step time."""
-    return world * dense_flops(wl) / (ms * 1e-3) / 1e12
+def job_value(wl, world: int, ms: float, sharded: bool = False) -> float:
+    """Whole-job effective TFLOP/s: the dense-equivalent FLOPs of all ranks
+    over the max-over-ranks step time (replicas: every rank its own
+    sequence; heads: the ranks share one sequence's heads)."""
+    return (1 if sharded else world) * dense_flops(wl) / (ms * 1e-3) / 1e12
 
 
 # ---------------------------------------------------------------- clocks
@@ -148,55 +182,74 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- oracle leg
-def oracle_sample(wl, tau: float, rows: int = 384, keep_recent: int = 0) -> dict:
+def oracle_sample(wl, tau: float, rows: int = 1536, heads: int = 2, keep_recent: int = 0) -> dict:
     """Time the CPU oracle on a bounded sample of the workload and scale it to
-    the whole step: steps 1-4 and 6 for one head at full length, step 5 for
-    the `rows` most expensive compressed rows of that head."""
+    the whole step: steps 1-4 and 6 at full length for the first `heads`
+    query heads of sequence 0 (their own KV heads), and step 5 for the `rows`
+    most expensive compressed rows of each.  The step estimate is the mean
+    per-head cost times the head count, with step 5 scaled by causal pairs."""
     import oracle as O
     try:
         from threadpoolctl import threadpool_info
         cores = max([t.get("num_threads", 1) for t in threadpool_info()] or [1])
     except Exception:  # pragma: no cover
         cores = 1
-    q, k, v = W.generate(wl.with_(B=1, Hq=1, Hkv=1))
+    heads = min(heads, wl.Hq)
+    sub = wl.with_(B=1, Hq=heads, Hkv=max(1, heads // wl.G) if heads >= wl.G else 1)
+    q, k, v = W.generate(sub)
+    G = sub.Hq // sub.Hkv
     L, d = wl.L, wl.d
     scale = O.default_scale(d)
-    t0 = time.perf_counter()
-    s32 = O.proxy_scores_head(q[0, 0, L - wl.w:], k[0, 0], L, scale)
-    kh = max(L - O.pruned_count_head(s32, tau), keep_recent)
-    sel = O.select_head(s32, kh, keep_recent)
-    qc, kc, vc = q[0, 0][sel], k[0, 0][sel], v[0, 0][sel]
-    t1 = time.perf_counter()
-    r = np.arange(kh - rows, kh)
-    oc = O.attention_rows(qc, kc, vc, r, scale)
-    t2 = time.perf_counter()
-    full = np.zeros((L, d))
-    full[sel[r]] = oc
-    t3 = time.perf_counter()
-    per_head_fixed = (t1 - t0) + (t3 - t2)
-    sample_pairs = float(np.sum(r + 1))
-    head_pairs = kh * (kh + 1) / 2.0
-    t_full = wl.B * wl.Hq * (per_head_fixed + (t2 - t1) * head_pairs / sample_pairs)
-    return {"seconds_full_step_est": t_full, "cores": cores, "sample_seconds": t3 - t0,
-            "k_head": int(kh),
-            "sample": (f"steps 1-4,6 for head (0,0) at L={L}, step 5 for its last {rows} compressed rows "
-                       f"(of k={kh}); scaled by head count and by causal pair count to the full step")}
+    fixed = attn = 0.0
+    pairs_sample = pairs_full = 0.0
+    ks = []
+    t_start = time.perf_counter()
+    for h in range(heads):
+        t0 = time.perf_counter()
+        s32 = O.proxy_scores_head(q[0, h, L - wl.w:], k[0, h // G], L, scale)
+        kh = max(L - O.pruned_count_head(s32, tau), keep_recent)
+        sel = O.select_head(s32, kh, keep_recent)
+        qc, kc, vc = q[0, h][sel], k[0, h // G][sel], v[0, h // G][sel]
+        t1 = time.perf_counter()
+        r = np.arange(max(kh - rows, 0), kh)
+        oc = O.attention_rows(qc, kc, vc, r, scale)
+        t2 = time.perf_counter()
+        full = np.zeros((L, d))
+        full[sel[r]] = oc
+        t3 = time.perf_counter()
+        fixed += (t1 - t0) + (t3 - t2)
+        attn += t2 - t1
+        pairs_sample += float(np.sum(r + 1))
+        pairs_full += kh * (kh + 1) / 2.0
+        ks.append(int(kh))
+    sample_seconds = time.perf_counter() - t_start
+    per_head = (fixed + attn * pairs_full / pairs_sample) / heads
+    t_full = wl.B * wl.Hq * per_head
+    return {"seconds_full_step_est": t_full, "cores": cores, "host_cores": len(os.sched_getaffinity(0)),
+            "sample_seconds": sample_seconds, "k_head": ks,
+            "sample": (f"steps 1-4,6 at L={L} for query heads 0..{heads - 1} of sequence 0, step 5 for the last "
+                       f"{rows} compressed rows of each (k={ks}); the mean per-head time scaled by head count, "
+                       f"step 5 by causal pair count, to the full step ({sample_seconds:.1f} s measured)")}
 
 
 def config_of(args, wl, world: int) -> dict:
     """The workload description both arms print."""
+    shard = getattr(args, "shard", "heads")
     return {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "L": wl.L, "d": wl.d, "w": wl.w,
             "tau": args.tau, "budget_mode": args.budget_mode, "keep_recent": args.keep_recent,
-            "layout": args.layout, "parallelism": f"replicas{world}" if world > 1 else "single",
+            "layout": args.layout, "parallelism": f"{shard}{world}" if world > 1 else "single",
             "l2": "inputs larger than L2 (Q 1 GiB, K/V 256 MiB each)"}
 
 
 def run_reference(args, wl, rank: int) -> int:
     if rank != 0:
         return 0
+    # each step a smaller sample (one head, 768 attention rows) so that the
+    # default --steps/--warmup run ends in a few minutes
+    one = lambda: oracle_sample(wl, args.tau, rows=768, heads=1, keep_recent=args.keep_recent)
     for _ in range(args.warmup):
-        oracle_sample(wl, args.tau, keep_recent=args.keep_recent)
-    runs = [oracle_sample(wl, args.tau, keep_recent=args.keep_recent) for _ in range(args.steps)]
+        one()
+    runs = [one() for _ in range(args.steps)]
     t = statistics.median(r["seconds_full_step_est"] for r in runs)
     value = dense_flops(wl) / t / 1e12
     line = {
@@ -204,8 +257,8 @@ def run_reference(args, wl, rank: int) -> int:
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_of(args, wl, args.gpus),
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": runs[0]["cores"], "kind": "oracle",
-                         "sample": runs[0]["sample"]},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": runs[0]["cores"], "host_cores": runs[0]["host_cores"],
+                         "kind": "oracle", "sample": runs[0]["sample"]},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -279,6 +332,101 @@ def run_varlen(args, wl) -> int:
     return 0
 
 
+# ---------------------------------------------------------------- sweep leg
+def run_sweep(args, wl) -> int:
+    """The forward over a grid of coverage thresholds and context lengths
+    (the workload's shape otherwise), one JSON line per point, on one GPU:
+    the forward's time, keep fraction, effective and achieved TFLOP/s, the
+    stage breakdown, and the dense baselines (our kernel and torch SDPA) on
+    the same tensors.  These are supporting lines, not the headline."""
+    import torch
+    import token_sparse_attention_tsa_b200 as T
+    T.load()
+    stream = torch.cuda.current_stream()
+    taus = [float(x) for x in args.sweep_tau.split(",")] if args.sweep_tau else [args.tau]
+    lengths = [int(x) for x in args.sweep_L.split(",")] if args.sweep_L else [wl.L]
+    pk = peaks()
+
+    def timed(fn, n):
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(n):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / n
+
+    for L in lengths:
+        wl_l = wl.with_(L=L, w=min(wl.w, L))
+        qh, kh, vh = W.generate(wl_l)
+        q, k, v = (torch.from_numpy(x).view(torch.bfloat16).cuda() for x in (qh, kh, vh))
+        del qh, kh, vh
+        o = torch.empty_like(q)
+        shape3 = (wl.B, wl.Hq, L)
+        scores = torch.empty(shape3, device="cuda")
+        idx = torch.empty(shape3, dtype=torch.int32, device="cuda")
+        k_seq = torch.empty((wl.B,), dtype=torch.int32, device="cuda")
+        k_head = torch.empty((wl.B, wl.Hq), dtype=torch.int32, device="cuda")
+        qc, kc, vc = (torch.empty((wl.B, wl.Hq, L, wl.d), dtype=torch.bfloat16, device="cuda") for _ in range(3))
+        p0 = T.params(wl.B, wl.Hq, wl.Hkv, L, wl.d, wl_l.w, taus[0])
+        ws = T.new_workspace(p0)
+        od = torch.empty_like(q)
+        T.tsa_attend_dense(p0, q, k, v, od, None, ws)
+        dense_ms = timed(lambda: T.tsa_attend_dense(p0, q, k, v, od, None, ws), 2)
+        sdpa_ms = None
+        try:
+            from torch.nn.attention import SDPBackend, sdpa_kernel
+            sdpa = torch.nn.functional.scaled_dot_product_attention
+            with sdpa_kernel([SDPBackend.CUDNN_ATTENTION, SDPBackend.FLASH_ATTENTION]):
+                sdpa(q, k, v, is_causal=True, enable_gqa=True)
+                sdpa_ms = timed(lambda: sdpa(q, k, v, is_causal=True, enable_gqa=True), 2)
+        except Exception:
+            sdpa_ms = None
+        for tau in taus:
+            p = T.params(wl.B, wl.Hq, wl.Hkv, L, wl.d, wl_l.w, tau)
+            fwd = lambda: T.tsa_forward(p, q, k, v, o, ws, scores, idx, k_seq)
+            for _ in range(args.warmup):
+                fwd()
+            with ClockSampler(0) as clk:
+                ms = timed(fwd, args.steps)
+            evs = [torch.cuda.Event(enable_timing=True) for _ in range(7)]
+            names = ["score", "budget", "select", "gather", "attend", "scatter"]
+            acc = {n: 0.0 for n in names}
+            reps = 2
+            for _ in range(reps):
+                evs[0].record(stream)
+                T.tsa_score(p, q, k, scores, ws); evs[1].record(stream)
+                T.tsa_budget(p, scores, k_head, k_seq, ws); evs[2].record(stream)
+                T.tsa_select(p, scores, k_seq, idx, ws); evs[3].record(stream)
+                T.tsa_gather_qkv(p, q, k, v, idx, k_seq, qc, kc, vc, ws); evs[4].record(stream)
+                T.tsa_attend(p, qc, kc, vc, k_seq, qc, None, ws); evs[5].record(stream)
+                T.tsa_scatter(p, qc, idx, k_seq, o, ws); evs[6].record(stream)
+                torch.cuda.synchronize()
+                for i, n in enumerate(names):
+                    acc[n] += evs[i].elapsed_time(evs[i + 1]) / reps
+            st = T.get_device_status(ws)
+            kept = k_seq.cpu().numpy()
+            cfl = compressed_flops(wl_l, kept)
+            line = {"metric": METRIC + " (sweep point)", "sweep": True, "n_gpus": 1, "steps": args.steps,
+                    "warmup": args.warmup, "dtype": "bf16", "data": "synthetic",
+                    "config": {"workload": wl.name, "L": L, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "d": wl.d,
+                               "w": wl_l.w, "tau": tau},
+                    "ms_per_step": ms, "k_seq": kept.tolist(), "keep_fraction": (kept / L).tolist(),
+                    "effective_tflops": dense_flops(wl_l) / (ms * 1e-3) / 1e12,
+                    "achieved_tflops": cfl / (ms * 1e-3) / 1e12,
+                    "attend_tflops": cfl / (acc["attend"] * 1e-3) / 1e12,
+                    "attend_frac_sustained": cfl / (acc["attend"] * 1e-3) / 1e12 / pk["bf16_sustained"],
+                    "dense_ms": dense_ms, "speedup_vs_dense": dense_ms / ms, "sdpa_dense_ms": sdpa_ms,
+                    "speedup_vs_sdpa": (sdpa_ms / ms) if sdpa_ms else None,
+                    "stage_ms": acc, "overhead_frac": (acc["score"] + acc["budget"] + acc["select"]) / acc["attend"],
+                    "status": st, "clocks": clk.summary()}
+            print(json.dumps(line), flush=True)
+        del q, k, v, o, qc, kc, vc, od, ws
+        torch.cuda.empty_cache()
+    return 0
+
+
 # ---------------------------------------------------------------- GPU leg
 def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
     import torch
@@ -302,9 +450,19 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
     def rank_max(x: float) -> float:
         return max_over_ranks(x, dist, dev)
 
-    # inputs: this rank's own sequence
-    wl_r = rank_workload(wl, rank)
-    qh, kh, vh = W.generate(wl_r)
+    # inputs: this rank's own sequence (replicas), or this rank's heads of
+    # the one sequence (heads: the same sequence on every rank, split by
+    # query head with the key/value heads they read)
+    sharded = world > 1 and args.shard == "heads"
+    if sharded:
+        h0, h1, kv0, kv1 = T.shard_heads(wl.Hq, wl.Hkv, world, rank)
+        qh, kh, vh = W.generate(wl)
+        qh, kh, vh = (np.ascontiguousarray(x[:, a:b]) for x, (a, b) in
+                      zip((qh, kh, vh), ((h0, h1), (kv0, kv1), (kv0, kv1))))
+        wl_all, wl = wl, wl.with_(Hq=h1 - h0, Hkv=kv1 - kv0)    # wl: this rank's part from here on
+    else:
+        wl_all = wl
+        qh, kh, vh = W.generate(rank_workload(wl, rank))
     if args.layout == "blhd":   # the caller's tensors token-major [B, L, H, d]
         qh, kh, vh = (np.ascontiguousarray(x.transpose(0, 2, 1, 3)) for x in (qh, kh, vh))
     pin = [torch.from_numpy(x).view(torch.bfloat16).pin_memory() for x in (qh, kh, vh)]
@@ -321,41 +479,54 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
     # or in the per-head mode each head's own count
     kept = k_head if args.budget_mode == "per_head" else k_seq
     shape = (wl.B, wl.Hq, wl.L, wl.d)
-    qc, kc, vc, oc = (torch.empty(shape, dtype=torch.bfloat16, device=dev) for _ in range(4))
+    qc, kc, vc = (torch.empty(shape, dtype=torch.bfloat16, device=dev) for _ in range(3))
     torch.cuda.synchronize()
 
-    def forward():
-        T.tsa_forward(p, q, k, v, o, ws, scores, idx, kept)
+    k_part = torch.empty((wl.B,), dtype=torch.int32, device=dev)
 
-    # the kernels tsa_forward runs, one ABI call each
-    stage_names = ["score", "budget", "select", "gather", "attend"]
+    def forward():
+        if sharded:   # steps 1-2 here, the budget exchanged over the ranks, steps 3-6 here
+            T.forward_sharded(p, wl_all.Hq, q, k, v, o, ws, scores_out=scores, idx_out=idx, k_seq_out=kept,
+                              k_part=k_part)
+        else:
+            T.tsa_forward(p, q, k, v, o, ws, scores, idx, kept)
+
+    # the kernels tsa_forward runs, one ABI call each (with head sharding, the
+    # budget's all-reduce over the ranks between the budget and the selection)
+    exchange_op = T.budget_reduce_op(args.budget_mode) if sharded else None
+    stage_names = ["score", "budget"] + (["exchange"] if exchange_op == "max" else []) + \
+        ["select", "gather", "attend", "scatter"]
 
     def staged(evs):
-        evs[0].record(stream)
+        n = iter(range(len(evs)))
+        evs[next(n)].record(stream)
         T.tsa_score(p, q, k, scores, ws)
-        evs[1].record(stream)
+        evs[next(n)].record(stream)
         T.tsa_budget(p, scores, k_head, k_seq, ws)
-        evs[2].record(stream)
+        evs[next(n)].record(stream)
+        if exchange_op == "max":
+            dist.all_reduce(k_seq, op=dist.ReduceOp.MAX)
+            evs[next(n)].record(stream)
         T.tsa_select(p, scores, kept, idx, ws)
-        evs[3].record(stream)
+        evs[next(n)].record(stream)
         T.tsa_gather_qkv(p, q, k, v, idx, kept, qc, kc, vc, ws)
-        evs[4].record(stream)
-        T.tsa_attend_scatter(p, qc, kc, vc, idx, kept, o, None, ws)
-        evs[5].record(stream)
+        evs[next(n)].record(stream)
+        T.tsa_attend(p, qc, kc, vc, kept, qc, None, ws)      # output over qc in place, as tsa_forward
+        evs[next(n)].record(stream)
+        T.tsa_scatter(p, qc, idx, kept, o, ws)
+        evs[next(n)].record(stream)
 
-    # the separate stage calls the fused attention replaces (attention into a
-    # compressed output, then the scatter), and the fully fused gathering
-    # variant, timed for comparison and the scatter's own HBM roofline
-    unfused_names = ["attend_compressed", "scatter", "attend_gathered"]
+    # the stage calls tsa_forward does not use, timed for comparison: the
+    # attention with the scatter folded into its epilogue (plus the zero fill
+    # of the unselected rows), and the variant that also gathers by index
+    unfused_names = ["attend_scatter_fused", "attend_gathered"]
 
     def unfused(evs):
         evs[0].record(stream)
-        T.tsa_attend(p, qc, kc, vc, kept, oc, None, ws)
+        T.tsa_attend_scatter(p, qc, kc, vc, idx, kept, o, None, ws)
         evs[1].record(stream)
-        T.tsa_scatter(p, oc, idx, kept, o, ws)
-        evs[2].record(stream)
         T.tsa_attend_gathered(p, q, k, v, idx, kept, o, None, ws)
-        evs[3].record(stream)
+        evs[2].record(stream)
 
     def timed(fn, n):
         barrier()
@@ -466,7 +637,11 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
             stream.wait_event(up)
             if i >= 2:
                 stream.wait_event(d2h_done[i - 2])         # this set's previous output is back on the host
-            T.tsa_forward(p, sq, sk, sv, so, ws, scores, idx, kept, stream=stream)
+            if sharded:
+                T.forward_sharded(p, wl_all.Hq, sq, sk, sv, so, ws, scores_out=scores, idx_out=idx, k_seq_out=kept,
+                                  k_part=k_part)
+            else:
+                T.tsa_forward(p, sq, sk, sv, so, ws, scores, idx, kept, stream=stream)
             comp_done[i] = torch.cuda.Event()
             comp_done[i].record(stream)
             d2h_s.wait_event(comp_done[i])
@@ -496,44 +671,48 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
     cflops = compressed_flops(wl, kept_np)
     attn_ms = stage_ms["attend"]
     achieved = cflops / (attn_ms * 1e-3) / 1e12
-    roof = {"bound": "tensor", "kernel": "attend2_kernel<128,false,true,false> (attention + scatter epilogue)",
+    roof = {"bound": "tensor", "kernel": "attend2_kernel<128,false,false,false> (attention, compressed output)",
             "achieved": achieved,
             "peak": pk["bf16_sustained"], "unit": "TFLOP/s", "frac": achieved / pk["bf16_sustained"],
-            "traffic": ATTN_DRAM_BYTES_PER_KEPT_ROW * kept_rows,
-            "traffic_note": "ncu DRAM bytes of one launch on the 32K workload, scaled by kept rows",
+            "traffic": (ATTN_DRAM_BYTES_PER_KEPT_ROW * kept_rows) if ATTN_DRAM_BYTES_PER_KEPT_ROW else None,
+            "traffic_note": ATTN_TRAFFIC_NOTE,
             "peak_note": f"bf16_tflops_sustained of {pk['source']} peaks (kernel timed inside a long step)"}
     hbm = pk["hbm_gbs"]
-    tok = wl.B * wl.Hq * wl.L
-    kept = kept_rows
-    stage_bytes = {
-        "gather": kept * wl.d * 2 * 3 * 2,                      # 3 rows read + 3 written
-        "scatter": tok * wl.d * 2 + kept * wl.d * 2,            # full write + kept rows read
-        "score": 2 * wl.B * wl.Hkv * wl.L * wl.d * 2 + tok * 4,  # two K passes + scores
-    }
-    times = {"gather": stage_ms["gather"], "scatter": unfused_ms["scatter"], "score": stage_ms["score"]}
-    stage_roof = {n: {"GB/s": b / (times[n] * 1e-3) / 1e9, "frac_hbm": b / (times[n] * 1e-3) / 1e9 / hbm}
+    stage_bytes = stage_algorithmic_bytes(wl, kept_np, idx)
+    times = {n: stage_ms[n] for n in stage_bytes}
+    stage_roof = {n: {"bytes": b, "GB/s": b / (times[n] * 1e-3) / 1e9, "frac_hbm": b / (times[n] * 1e-3) / 1e9 / hbm}
                   for n, b in stage_bytes.items()}
+    # the proxy score is bound by its exponentials: 2 B Hq w L of them (two passes)
+    exps = 2.0 * wl.B * wl.Hq * wl.w * wl.L
+    ex2_peak = EX2_PER_CLK_SM * SMS * (clocks.get("sm_mhz") or 1965.0) * 1e6
+    stage_roof["score"]["exp_per_s"] = exps / (stage_ms["score"] * 1e-3)
+    stage_roof["score"]["exp_frac"] = stage_roof["score"]["exp_per_s"] / ex2_peak
+    stage_roof["score"]["exp_peak_note"] = (f"{EX2_PER_CLK_SM} ex2/clk/SM x {SMS} SMs x the median sampled SM clock "
+                                            "(ex2.approx rate of one warp instruction per 4 clocks per SMSP)")
 
-    value = job_value(wl, world, ms)
+    job_flops = dense_flops(wl_all) * (1 if sharded else world)   # the work of all ranks together
+    value = job_value(wl_all, world, ms, sharded)
     cpu = None
     if rank == 0 and not args.no_cpu_baseline:
-        s = oracle_sample(wl, args.tau, keep_recent=args.keep_recent)
-        cpu = {"value": dense_flops(wl) / s["seconds_full_step_est"] / 1e12, "unit": UNIT, "cores": s["cores"],
-               "kind": "oracle", "sample": s["sample"], "sample_seconds": s["sample_seconds"]}
+        s = oracle_sample(wl_all, args.tau, keep_recent=args.keep_recent)
+        cpu = {"value": dense_flops(wl_all) / s["seconds_full_step_est"] / 1e12, "unit": UNIT,
+               "cores": s["cores"], "host_cores": s["host_cores"], "kind": "oracle", "sample": s["sample"],
+               "sample_seconds": s["sample_seconds"]}
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+        "scaling": "strong" if sharded else "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": config_of(args, wl, world),
+        "config": config_of(args, wl_all, world),
         "k_seq": ks, "keep_fraction": [x / wl.L for x in ks],
         "kept_fraction_all_heads": kept_rows / float(wl.B * wl.Hq * wl.L),
         "dense_ms": dense_ms, "speedup_vs_dense": dense_ms / ms, "sdpa_dense_ms": sdpa_ms,
-        "effective_tflops": dense_flops(wl) / (ms * 1e-3) / 1e12,
-        "achieved_tflops": cflops / (ms * 1e-3) / 1e12,
+        "effective_tflops": value,
+        "achieved_tflops": cflops / (ms * 1e-3) / 1e12 * (world if sharded else 1),
         "stage_ms": stage_ms, "unfused_stage_ms": unfused_ms, "stage_hbm": stage_roof,
         "overhead_frac": (sum(stage_ms.values()) - attn_ms) / attn_ms,
         "roofline": roof, "cpu_baseline": cpu,
-        "e2e": {"value": job_value(wl, world, e2e_ms), "unit": UNIT, "ms_per_step": e2e_ms,
+        "e2e": {"value": job_flops / (e2e_ms * 1e-3) / 1e12, "unit": UNIT, "ms_per_step": e2e_ms,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                 "note": "every step copies its inputs up and its output back; copies of neighbouring steps "
                         "overlap this step's compute on separate streams (pipeline fill and drain included)"},
@@ -561,12 +740,18 @@ def main() -> int:
     ap.add_argument("--budget-mode", default="max", choices=["max", "mean", "per_head"])
     ap.add_argument("--keep-recent", type=int, default=0)
     ap.add_argument("--layout", default="bhld", choices=["bhld", "blhd"])
+    ap.add_argument("--shard", default="heads", choices=["heads", "replicas"],
+                    help="with --gpus N > 1: split the query heads of the one sequence over the ranks (one "
+                         "all-reduce of the budget per step; strong scaling), or give every rank its own "
+                         "sequence (no collective; weak scaling)")
     ap.add_argument("--blocks", default=None,
                     help="band:N -- also time the path with a block-sparse mask on the compressed sequence "
                          "(sink block + local band of N blocks)")
     ap.add_argument("--varlen", default=None,
                     help="comma-separated sequence lengths: time a packed varlen batch of the workload's "
                          "first L_b tokens per sequence instead of the headline step")
+    ap.add_argument("--sweep-tau", default=None, help="comma-separated tau values: print one sweep line each")
+    ap.add_argument("--sweep-L", default=None, help="comma-separated context lengths for the sweep")
     args = ap.parse_args()
     wl = W.WORKLOADS[args.workload]
     if args.tau is None:
@@ -579,6 +764,8 @@ def main() -> int:
         return run_reference(args, wl, rank)
     if args.varlen:
         return run_varlen(args, wl)
+    if args.sweep_tau or args.sweep_L:
+        return run_sweep(args, wl)
     return run_gpu(args, wl, rank, world, local_rank)
 
 

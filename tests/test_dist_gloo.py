@@ -1,9 +1,10 @@
 """The multi-rank host logic of bench.py, run as two gloo ranks on CPU.
 
-The path shards by sequence: each rank processes its own sequence and no data
-crosses ranks.  What the ranks share is the job's clock: the step time is the
-max over ranks and the value sums every rank's work.  These tests check that
-logic (and the per-rank inputs) without a GPU.
+With --shard replicas each rank processes its own sequence and no data
+crosses ranks; with --shard heads (tests/test_dist_shard_heads.py) the ranks
+split one sequence's heads.  Either way the ranks share the job's clock: the
+step time is the max over ranks, and the value counts the work of the whole
+job.  These tests check that logic (and the per-rank inputs) without a GPU.
 """
 import os
 import socket
@@ -70,6 +71,8 @@ def test_job_value_sums_ranks():
     one = bench.job_value(wl, 1, 100.0)
     assert abs(one - bench.dense_flops(wl) / 0.1 / 1e12) < 1e-9
     assert abs(bench.job_value(wl, 8, 100.0) - 8 * one) < 1e-6
+    # heads of one sequence split over 8 ranks: the job is that one sequence
+    assert abs(bench.job_value(wl, 8, 100.0, sharded=True) - one) < 1e-9
     assert bench.max_over_ranks(3.5, None, None) == 3.5
 
 
@@ -104,4 +107,31 @@ def test_both_arms_print_the_same_config():
     args = argparse.Namespace(tau=0.05, budget_mode="max", keep_recent=0, layout="bhld", gpus=1)
     cfg = bench.config_of(args, wl, 1)
     assert cfg["workload"] == "c4_L128K_gqa" and cfg["L"] == 131072 and cfg["parallelism"] == "single"
+    assert bench.config_of(args, wl, 4)["parallelism"] == "heads4"      # the default split
+    args.shard = "replicas"
     assert bench.config_of(args, wl, 4)["parallelism"] == "replicas4"
+
+
+def test_stage_bytes_count_unique_kv_rows_per_group():
+    """The gather's algorithmic bytes count each K/V row a KV group reads once
+    (the union of its query heads' selections), per the measurement plan."""
+    import sys
+
+    import numpy as np
+    import torch
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads as W
+    wl = W.WORKLOADS["c1_L1K_mha_d64"].with_(B=1, Hq=4, Hkv=2, L=8, d=64, w=2)
+    idx = torch.full((1, 4, 8), -1, dtype=torch.int32)
+    sel = {0: [0, 1, 2], 1: [1, 2, 3], 2: [5, 6, 7], 3: [5, 6, 7]}   # group 0 reads 4 rows, group 1 reads 3
+    for h, s in sel.items():
+        idx[0, h, :3] = torch.tensor(s)
+    b = bench.stage_algorithmic_bytes(wl, np.array([3]), idx)
+    row = 64 * 2
+    assert b["gather"] == 12 * row + 2 * 7 * row + 3 * 12 * row
+    assert b["scatter"] == 4 * 8 * row + 12 * row
+    assert b["score"] == 2 * 8 * row + 4 * 2 * row + 4 * 8 * 4
+    # per-head counts: head 3 keeps only 2 rows, so group 1 still reads rows 5, 6, 7 (head 2)
+    b2 = bench.stage_algorithmic_bytes(wl, np.array([[3, 3, 3, 2]]), idx)
+    assert b2["gather"] == 11 * row + 2 * 7 * row + 3 * 11 * row

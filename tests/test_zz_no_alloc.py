@@ -73,8 +73,9 @@ def test_noalloc_reports_a_timeout_and_the_next_call_is_clean():
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
-    # scratch here: 64 heads x 4096 window rows x 4096 key chunks x 12 bytes, far over 16 MiB
-    p = T.params(1, 64, 8, 1 << 22, 128, 4096, 0.05)
+    # scratch here: 8 x 64 heads x 4096 window rows x (12 bytes per key chunk + 8 bytes of row
+    # statistics), over 40 MB, far beyond the 16 MiB array
+    p = T.params(8, 64, 8, 1 << 21, 128, 4096, 0.05)
     assert T.stage_workspace_size(p) > T.NOALLOC_SCRATCH_BYTES
     q = torch.empty(16, dtype=torch.bfloat16, device="cuda")   # never touched: rejected on the host
     s = torch.empty(4, dtype=torch.float32, device="cuda")

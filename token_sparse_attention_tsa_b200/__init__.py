@@ -371,16 +371,19 @@ def shard_heads(Hq: int, Hkv: int, world: int, rank: int) -> tuple[int, int, int
     return h0, h1, h0 // G, (h1 - 1) // G + 1
 
 
-def forward_sharded(p, Hq_total: int, q, k, v, o, ws, group=None, scores_out=None, idx_out=None, k_seq_out=None):
+def forward_sharded(p, Hq_total: int, q, k, v, o, ws, group=None, scores_out=None, idx_out=None, k_seq_out=None,
+                    k_part=None):
     """The forward of this device's heads of a head-sharded batch (p, q, k, v,
     o describe the local heads; Hq_total counts a sequence's query heads over
     all devices): tsa_forward_begin, one all-reduce of the B budget partials
     over `group` (torch.distributed, e.g. NCCL; skipped when nothing is
     shared or the group has one member), tsa_forward_end.  Runs on the
-    current CUDA stream."""
+    current CUDA stream.  k_part: optional int32 [B] buffer for the partials
+    (allocated when None); returned after the exchange."""
     import torch
     import torch.distributed as dist
-    k_part = torch.empty((p.B,), dtype=torch.int32, device=q.device)
+    if k_part is None:
+        k_part = torch.empty((p.B,), dtype=torch.int32, device=q.device)
     tsa_forward_begin(p, q, k, k_part, ws, scores_out=scores_out)
     op = budget_reduce_op(p.budget_mode)
     if op is not None and dist.is_available() and dist.is_initialized() and dist.get_world_size(group) > 1:

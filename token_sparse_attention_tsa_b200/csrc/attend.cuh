@@ -23,6 +23,14 @@
 
 namespace tsa {
 
+// Pairs e (of the 16 value pairs of each 32-column chunk of a softmax row)
+// whose two exponentials are computed by exp2_poly_x2 on the FMA pipe; the
+// others use ex2.approx on the MUFU unit.  The split balances the two units.
+#ifndef TSA_EXP_EMU_PAIRS
+#define TSA_EXP_EMU_PAIRS 0x0000u
+#endif
+constexpr uint32_t kExpEmuPairs = TSA_EXP_EMU_PAIRS;
+
 struct AttnArgs {
   Kept kept;              // valid rows per (b, h) (null counts: L)
   __nv_bfloat16* o;       // B x Hq heads of L rows of D
@@ -455,10 +463,16 @@ __global__ void __launch_bounds__(Attn2Layout<D>::THREADS, 1)
           uint32_t (&pk)[16] = *reinterpret_cast<uint32_t(*)[16]>(&pk32[kWide ? cc * 16 : 0]);
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            float x0, x1;
-            f2_unpack(f2_fma(f2_pack(sv[c][2 * e], sv[c][2 * e + 1]), sl2x2, nmx2), x0, x1);
-            const float p0 = ex2_approx(x0);
-            const float p1 = ex2_approx(x1);
+            const uint64_t xx = f2_fma(f2_pack(sv[c][2 * e], sv[c][2 * e + 1]), sl2x2, nmx2);
+            float p0, p1;
+            if ((kExpEmuPairs >> e) & 1u) {            // this pair on the FMA pipe
+              exp2_poly_x2(xx, p0, p1);
+            } else {                                   // this pair on the MUFU unit
+              float x0, x1;
+              f2_unpack(xx, x0, x1);
+              p0 = ex2_approx(x0);
+              p1 = ex2_approx(x1);
+            }
             r4[e & 3] = f2_add(r4[e & 3], f2_pack(p0, p1));
             pk[e] = pack_bf16x2(p0, p1);
           }

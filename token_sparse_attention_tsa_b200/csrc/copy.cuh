@@ -27,41 +27,70 @@ struct GatherArgs {
   Seqs seqs;                       // sequence lengths L_b
   __nv_bfloat16 *qc, *kc, *vc;     // [B*Hq, L, D]; qc may be null (K and V only)
   uint32_t* status;                // or null
-  int L, Hq, Hkv, G;
-  long long total_rows;            // B*Hq*L
+  int B, L, Hq, Hkv, G;
 };
 
+constexpr int GT_ROWS = 32;        // compressed rows per gather work item (per query head)
+
+// Work item: (sequence b, KV head g, GT_ROWS compressed rows i) for all G
+// query heads of the group, rows visited with the query head fastest: the
+// G heads copy their i-th selected rows back to back.  Their selections
+// ascend and overlap heavily, so the K and V rows they read are close
+// together and come from L2 after the first head's read: each K/V row
+// crosses HBM about once per group rather than once per query head.  Index
+// arithmetic is 32-bit and done once per item; each thread keeps two rows'
+// loads in flight.
 template <int D>
-__global__ void __launch_bounds__(256) gather_kernel(const GatherArgs a) {
-  constexpr int LPR = D / 8;  // lanes per row
+__global__ void __launch_bounds__(256, 4) gather_kernel(const GatherArgs a) {
+  constexpr int LPR = D / 8;       // lanes per row
+  constexpr int RPP = 256 / LPR;   // rows per pass of the CTA
   const int sub = threadIdx.x % LPR;
-  const long long stride = static_cast<long long>(gridDim.x) * (blockDim.x / LPR);
+  const int slot = threadIdx.x / LPR;
+  const int tiles = (a.L + GT_ROWS - 1) / GT_ROWS;
+  const int items = a.B * a.Hkv * tiles;
+  const int per_item = GT_ROWS * a.G;
   bool bad = false;
-  for (long long row = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) / LPR;
-       row < a.total_rows; row += stride) {
-    const long long bh = row / a.L;
-    const int i = static_cast<int>(row - bh * a.L);
-    const int b = static_cast<int>(bh / a.Hq);
-    const int h = static_cast<int>(bh - static_cast<long long>(b) * a.Hq);
+  for (int w = blockIdx.x; w < items; w += gridDim.x) {
+    const int bg = w / tiles, tile = w - bg * tiles;
+    const int b = bg / a.Hkv, g = bg - b * a.Hkv;
     const int Lb = a.seqs.len(b);
-    if (i >= a.kept.of(b, h, Lb)) continue;
-    const int j = __ldg(a.idx + row);
-    const size_t dst = static_cast<size_t>(row) * D + sub * 8;
-    if (j < 0 || j >= Lb) {
-      bad = true;
-      const uint4 z = make_uint4(0, 0, 0, 0);
-      if (a.qc) *reinterpret_cast<uint4*>(a.qc + dst) = z;
-      *reinterpret_cast<uint4*>(a.kc + dst) = z;
-      *reinterpret_cast<uint4*>(a.vc + dst) = z;
-      continue;
+    const int i0 = tile * GT_ROWS;
+    if (i0 >= Lb) continue;
+    for (int r0 = slot; r0 < per_item; r0 += 2 * RPP) {
+      int h[2], i[2], j[2];
+      bool live[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int r = r0 + u * RPP;
+        const int di = r / a.G;
+        i[u] = i0 + di;
+        h[u] = g * a.G + (r - di * a.G);
+        live[u] = r < per_item && i[u] < a.kept.of(b, h[u], Lb);
+        j[u] = live[u] ? __ldg(a.idx + (static_cast<size_t>(b) * a.Hq + h[u]) * a.L + i[u]) : 0;
+      }
+      uint4 vq[2], vk[2], vv[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        vq[u] = vk[u] = vv[u] = make_uint4(0, 0, 0, 0);
+        const bool ok = j[u] >= 0 && j[u] < Lb;
+        bad |= live[u] && !ok;           // a bad index: a zero row, reported
+        if (live[u] && ok) {
+          const size_t skv = a.kvs.at(b, g, j[u]) + sub * 8;
+          vk[u] = __ldg(reinterpret_cast<const uint4*>(a.k + skv));
+          vv[u] = __ldg(reinterpret_cast<const uint4*>(a.v + skv));
+          if (a.qc) vq[u] = __ldg(reinterpret_cast<const uint4*>(a.q + a.qs.at(b, h[u], j[u]) + sub * 8));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        if (live[u]) {
+          const size_t dst = ((static_cast<size_t>(b) * a.Hq + h[u]) * a.L + i[u]) * D + sub * 8;
+          if (a.qc) *reinterpret_cast<uint4*>(a.qc + dst) = vq[u];
+          *reinterpret_cast<uint4*>(a.kc + dst) = vk[u];
+          *reinterpret_cast<uint4*>(a.vc + dst) = vv[u];
+        }
+      }
     }
-    const size_t sq = a.qs.at(b, h, j) + sub * 8;
-    const size_t skv = a.kvs.at(b, h / a.G, j) + sub * 8;
-    const uint4 vk = __ldg(reinterpret_cast<const uint4*>(a.k + skv));
-    const uint4 vv = __ldg(reinterpret_cast<const uint4*>(a.v + skv));
-    if (a.qc) *reinterpret_cast<uint4*>(a.qc + dst) = __ldg(reinterpret_cast<const uint4*>(a.q + sq));
-    *reinterpret_cast<uint4*>(a.kc + dst) = vk;
-    *reinterpret_cast<uint4*>(a.vc + dst) = vv;
   }
   if (bad && a.status) atomicOr(a.status, 0x4u);
 }

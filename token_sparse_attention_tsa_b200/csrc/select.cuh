@@ -18,10 +18,15 @@
 // maximum is the default reading; the mean and a per-head budget (every
 // head keeps its own k_head) are the two other plain readings, selectable.
 // Ascending order of q_j is the ascending order of the fp32 bit patterns, so
-// neither kernel sorts: both run a most-significant-digit radix descent
-// (4 levels of 8 bits) over the score bit patterns with per-warp shared
-// histograms, then (select) compact the chosen indices in index order, which
-// yields S_h ascending.  Ties at the threshold go to the smaller index.
+// neither kernel sorts: both run a most-significant-digit radix descent over
+// the bit patterns, then (select) compact the chosen indices in index order,
+// which yields S_h ascending.  Ties at the threshold go to the smaller index.
+// The descent runs on r = key - min_key with 11-bit digits taken from the top
+// of the head's own key range (at most three levels), after one pass that
+// finds the range: the scores of a head span a few binary orders of
+// magnitude, so digits of the raw bit pattern's top bits would put nearly
+// every key of a warp into the same few bins and serialise the shared-memory
+// histogram atomics.
 #pragma once
 
 #include <cstdint>
@@ -69,34 +74,114 @@ __device__ __forceinline__ T block_sum(T v, T* red) {
 }
 
 // Exclusive prefix sum over the block (thread order); returns the total too.
-__device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, uint32_t* red, uint32_t& total) {
+// red: at least 33 entries of shared memory.
+template <typename T>
+__device__ __forceinline__ T block_exclusive_scan(T v, T* red, T& total) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  uint32_t inc = v;
+  T inc = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const uint32_t y = __shfl_up_sync(0xffffffffu, inc, o);
+    const T y = __shfl_up_sync(0xffffffffu, inc, o);
     if (lane >= o) inc += y;
   }
   __syncthreads();
   if (lane == 31) red[warp] = inc;
   __syncthreads();
   if (warp == 0) {
-    uint32_t x = red[lane];
-    uint32_t xi = x;
+    const T x = lane < BS_WARPS ? red[lane] : T(0);
+    T xi = x;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(0xffffffffu, xi, o);
+      const T y = __shfl_up_sync(0xffffffffu, xi, o);
       if (lane >= o) xi += y;
     }
     red[lane] = xi - x;       // exclusive prefix of warp totals
     if (lane == 31) red[32] = xi;
   }
   __syncthreads();
-  const uint32_t r = red[warp] + inc - v;
+  const T r = red[warp] + inc - v;
   total = red[32];
   __syncthreads();
   return r;
 }
+
+// Block-wide minimum and maximum of u32 values (red: at least 2 * 32 entries).
+__device__ __forceinline__ void block_minmax(uint32_t& mn, uint32_t& mx, uint32_t* red) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  mn = __reduce_min_sync(0xffffffffu, mn);
+  mx = __reduce_max_sync(0xffffffffu, mx);
+  __syncthreads();
+  if (lane == 0) {
+    red[warp] = mn;
+    red[32 + warp] = mx;
+  }
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t a = lane < BS_WARPS ? red[lane] : 0xffffffffu;
+    uint32_t b = lane < BS_WARPS ? red[32 + lane] : 0u;
+    a = __reduce_min_sync(0xffffffffu, a);
+    b = __reduce_max_sync(0xffffffffu, b);
+    if (lane == 0) {
+      red[0] = a;
+      red[32] = b;
+    }
+  }
+  __syncthreads();
+  mn = red[0];
+  mx = red[32];
+  __syncthreads();
+}
+
+// Visit scores sc[j] for j = threadIdx.x, +1024, ... below n, loading BATCH
+// of them before using any: one CTA per head walks a 4L-byte row several
+// times, and with one load in flight per thread the walk is bound by L2
+// latency, not bandwidth.  f(j, value) is called in index order per thread.
+constexpr int BS_BATCH = 8;
+template <typename F>
+__device__ __forceinline__ void for_each_score(const float* __restrict__ sc, int n, F&& f) {
+  for (int j0 = threadIdx.x; j0 < n; j0 += BS_THREADS * BS_BATCH) {
+    float v[BS_BATCH];
+#pragma unroll
+    for (int u = 0; u < BS_BATCH; ++u) {
+      const int j = j0 + u * BS_THREADS;
+      v[u] = j < n ? __ldg(sc + j) : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < BS_BATCH; ++u) {
+      const int j = j0 + u * BS_THREADS;
+      if (j < n) f(j, v[u]);
+    }
+  }
+}
+
+constexpr int RD_BITS = 11;                 // digit width of the radix descent
+constexpr int RD_BINS = 1 << RD_BITS;       // 2048 bins per level
+constexpr int BUD_COPIES = 4;               // budget histogram copies (eight warps each)
+constexpr int SEL_COPIES = 8;               // select histogram copies (four warps each)
+constexpr int BUD_SMEM = BUD_COPIES * RD_BINS * (8 + 4);
+constexpr int SEL_SMEM = SEL_COPIES * RD_BINS * 4;
+
+// Digit plan of a descent over r = key - kmin: nb is the bit length of
+// kmax - kmin; level l covers bits [lo(l), hi(l)) of r, 11 bits at a time
+// from the top, and the last level ends at bit 0.  An element takes part in
+// level l when its bits above hi(l) equal the prefix chosen so far.
+struct DigitPlan {
+  uint32_t kmin;
+  int nb;
+  __device__ __forceinline__ int levels() const { return nb <= RD_BITS ? 1 : (nb + RD_BITS - 1) / RD_BITS; }
+  __device__ __forceinline__ int hi(int l) const { return nb - RD_BITS * l; }
+  __device__ __forceinline__ int lo(int l) const {
+    const int x = nb - RD_BITS * (l + 1);
+    return x < 0 ? 0 : x;
+  }
+  // digit of key u at level l, or -1 when it is not a candidate there
+  __device__ __forceinline__ int digit(uint32_t u, int l, uint32_t prefix) const {
+    const uint32_t r = u - kmin;
+    const int h = hi(l), w = h - lo(l);
+    if ((static_cast<uint64_t>(r) >> h) != prefix) return -1;
+    return static_cast<int>((r >> lo(l)) & ((1u << w) - 1u));
+  }
+};
 
 struct BudgetArgs {
   const float* scores;  // [B*Hq, L]: the first L_b entries of each row are read
@@ -108,93 +193,94 @@ struct BudgetArgs {
   Seqs seqs;            // sequence lengths L_b
 };
 
-// grid: B*Hq CTAs of 1024 threads; dynamic smem: per-warp histograms.
+// grid: B*Hq CTAs of 1024 threads; dynamic smem: BUD_SMEM (count and mass
+// histograms, BUD_COPIES copies).
 __global__ void __launch_bounds__(BS_THREADS, 1) budget_kernel(const BudgetArgs a) {
   extern __shared__ __align__(16) uint8_t bsm[];
-  unsigned long long* hsum = reinterpret_cast<unsigned long long*>(bsm);             // [32][256]
-  uint32_t* hcnt = reinterpret_cast<uint32_t*>(bsm + BS_WARPS * 256 * 8);            // [32][256]
-  __shared__ unsigned long long red64[BS_WARPS];
+  unsigned long long* hsum = reinterpret_cast<unsigned long long*>(bsm);           // [copies][bins]
+  uint32_t* hcnt = reinterpret_cast<uint32_t*>(bsm + BUD_COPIES * RD_BINS * 8);    // [copies][bins]
+  __shared__ unsigned long long red64[33];
+  __shared__ uint32_t red32[64];
   __shared__ unsigned long long s_rem;
-  __shared__ uint32_t s_below, s_prefix, s_mask, s_done;
+  __shared__ uint32_t s_below, s_chosen;
 
   const int bh = blockIdx.x;
   const float* sc = a.scores + static_cast<size_t>(bh) * a.L;
-  const int warp = threadIdx.x >> 5;
+  const int copy = (threadIdx.x >> 5) % BUD_COPIES;
   bool bad = false, bad_seq = false;
   const int Lb = a.seqs.len_ok(bh / a.Hq, bad_seq);
 
+  // pass 0: total mass and the key range
   unsigned long long tot = 0;
-  for (int j = threadIdx.x; j < Lb; j += BS_THREADS) tot += mass_of_key(score_key(sc[j], bad));
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+  for_each_score(sc, Lb, [&](int, float x) {
+    const uint32_t u = score_key(x, bad);
+    tot += mass_of_key(u);
+    kmin = min(kmin, u);
+    kmax = max(kmax, u);
+  });
   tot = block_sum<unsigned long long>(tot, red64);
+  block_minmax(kmin, kmax, red32);
   const unsigned long long T =
       static_cast<unsigned long long>(floor(__dmul_rn(a.tau, __ull2double_rn(tot))));
-  if (threadIdx.x == 0) {
-    s_rem = T;
-    s_below = 0;
-    s_prefix = 0;
-    s_mask = 0;
-    s_done = 0;
-  }
-  __syncthreads();
-
-  for (int level = 0; level < 4; ++level) {
-    const int shift = 24 - 8 * level;
-    for (int i = threadIdx.x; i < BS_WARPS * 256; i += BS_THREADS) {
+  const DigitPlan plan{kmin, Lb > 0 ? 32 - __clz(static_cast<int>(kmax - kmin)) : 0};
+  unsigned long long rem = T;
+  uint32_t below = 0, prefix = 0;
+  bool done = Lb == 0;
+  for (int l = 0; !done && l < plan.levels(); ++l) {
+    for (int i = threadIdx.x; i < BUD_COPIES * RD_BINS; i += BS_THREADS) {
       hsum[i] = 0;
       hcnt[i] = 0;
     }
     __syncthreads();
-    const uint32_t prefix = s_prefix, mask = s_mask;
-    for (int j = threadIdx.x; j < Lb; j += BS_THREADS) {
-      const uint32_t u = score_key(sc[j], bad);
-      if ((u & mask) == prefix) {
-        const uint32_t dgt = (u >> shift) & 255u;
-        atomicAdd(&hcnt[warp * 256 + dgt], 1u);
-        atomicAdd(&hsum[warp * 256 + dgt], static_cast<unsigned long long>(mass_of_key(u)));
+    for_each_score(sc, Lb, [&](int, float x) {
+      const uint32_t u = score_key(x, bad);
+      const int dg = plan.digit(u, l, prefix);
+      if (dg >= 0) {
+        atomicAdd(&hcnt[copy * RD_BINS + dg], 1u);
+        atomicAdd(&hsum[copy * RD_BINS + dg], static_cast<unsigned long long>(mass_of_key(u)));
       }
+    });
+    __syncthreads();
+    // thread t owns bins 2t and 2t+1 (ascending key order)
+    unsigned long long s2[2] = {0, 0}, c2[2] = {0, 0};
+#pragma unroll
+    for (int e = 0; e < 2; ++e)
+#pragma unroll
+      for (int c = 0; c < BUD_COPIES; ++c) {
+        s2[e] += hsum[c * RD_BINS + 2 * threadIdx.x + e];
+        c2[e] += hcnt[c * RD_BINS + 2 * threadIdx.x + e];
+      }
+    unsigned long long tot_s, tot_c;
+    const unsigned long long es = block_exclusive_scan<unsigned long long>(s2[0] + s2[1], red64, tot_s);
+    const unsigned long long ec = block_exclusive_scan<unsigned long long>(c2[0] + c2[1], red64, tot_c);
+    if (tot_s <= rem) {        // every candidate fits under the threshold: all are pruned
+      below += static_cast<uint32_t>(tot_c);
+      done = true;
+      break;
+    }
+    // the one bin where the running mass first exceeds rem: bins before it
+    // are pruned whole, bins after it are kept whole
+    if (es <= rem && rem < es + s2[0]) {
+      s_chosen = 2 * threadIdx.x;
+      s_rem = rem - es;
+      s_below = below + static_cast<uint32_t>(ec);
+    } else if (es + s2[0] <= rem && rem < es + s2[0] + s2[1]) {
+      s_chosen = 2 * threadIdx.x + 1;
+      s_rem = rem - es - s2[0];
+      s_below = below + static_cast<uint32_t>(ec + c2[0]);
     }
     __syncthreads();
-    if (threadIdx.x < 256) {
-      unsigned long long s = 0;
-      uint32_t c = 0;
-      for (int w = 0; w < BS_WARPS; ++w) {
-        s += hsum[w * 256 + threadIdx.x];
-        c += hcnt[w * 256 + threadIdx.x];
-      }
-      hsum[threadIdx.x] = s;
-      hcnt[threadIdx.x] = c;
-    }
+    rem = s_rem;
+    below = s_below;
+    prefix = (prefix << (plan.hi(l) - plan.lo(l))) | s_chosen;
     __syncthreads();
-    if (threadIdx.x == 0) {
-      unsigned long long rem = s_rem;
-      uint32_t below = s_below;
-      int chosen = -1;
-      for (int dgt = 0; dgt < 256; ++dgt) {
-        if (hsum[dgt] <= rem) {
-          rem -= hsum[dgt];
-          below += hcnt[dgt];
-        } else {
-          chosen = dgt;
-          break;
-        }
-      }
-      s_rem = rem;
-      s_below = below;
-      if (chosen < 0) {
-        s_done = 1;  // everything left fits under T
-      } else {
-        s_prefix = prefix | (static_cast<uint32_t>(chosen) << shift);
-        s_mask = mask | (255u << shift);
-      }
-    }
-    __syncthreads();
-    if (s_done) break;
   }
   if (threadIdx.x == 0) {
-    uint32_t p = s_below;
-    if (!s_done) {
-      const unsigned long long qstar = mass_of_key(s_prefix);  // > 0 here
-      p += static_cast<uint32_t>(s_rem / qstar);
+    uint32_t p = below;
+    if (!done) {  // the descent ended on one key value: its tokens share one mass
+      const unsigned long long qstar = mass_of_key(kmin + prefix);   // > 0 here
+      p += static_cast<uint32_t>(rem / qstar);
     }
     const int32_t kh = Lb - static_cast<int32_t>(p);
     const int32_t r = a.keep_recent < Lb ? a.keep_recent : Lb;
@@ -255,12 +341,14 @@ __device__ __forceinline__ uint32_t select_key(float s, int j, int first_forced,
   return j >= first_forced ? 0xffffffffu : u;
 }
 
-// grid: B*Hq CTAs of 1024 threads; dynamic smem: per-warp count histograms.
+// grid: B*Hq CTAs of 1024 threads; dynamic smem: SEL_SMEM (count
+// histograms, SEL_COPIES copies).
 __global__ void __launch_bounds__(BS_THREADS, 1) select_kernel(const SelectArgs a) {
   extern __shared__ __align__(16) uint8_t ssm[];
-  uint32_t* hcnt = reinterpret_cast<uint32_t*>(ssm);  // [32][256]
-  __shared__ uint32_t red[33];
-  __shared__ uint32_t s_rem, s_prefix, s_mask;
+  uint32_t* hcnt = reinterpret_cast<uint32_t*>(ssm);  // [copies][bins]
+  __shared__ uint32_t red[64];
+  __shared__ uint32_t s_rem, s_chosen;
+  __shared__ uint32_t w_gt[BS_WARPS], w_eq[BS_WARPS], w_base[BS_WARPS], w_eqb[BS_WARPS];
 
   const int bh = blockIdx.x;
   const int cap = a.L;                               // row capacity of idx
@@ -269,7 +357,8 @@ __global__ void __launch_bounds__(BS_THREADS, 1) select_kernel(const SelectArgs 
   int32_t* out = a.idx + static_cast<size_t>(bh) * cap;
   const int k = a.kept.of(bh / a.Hq, bh % a.Hq, L);
   const int first_forced = L - (a.keep_recent < L ? a.keep_recent : L);
-  const int warp = threadIdx.x >> 5;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int copy = warp % SEL_COPIES;
   bool bad = false;
 
   if (k == L) {  // everything kept
@@ -280,74 +369,118 @@ __global__ void __launch_bounds__(BS_THREADS, 1) select_kernel(const SelectArgs 
     for (int i = threadIdx.x; i < cap; i += BS_THREADS) out[i] = -1;
     return;
   }
-  if (threadIdx.x == 0) {
-    s_rem = static_cast<uint32_t>(k);
-    s_prefix = 0;
-    s_mask = 0;
+  // pass 0: the key range
+  uint32_t kmin = 0xffffffffu, kmax = 0u;
+  for_each_score(sc, L, [&](int j, float x) {
+    const uint32_t u = select_key(x, j, first_forced, bad);
+    kmin = min(kmin, u);
+    kmax = max(kmax, u);
+  });
+  block_minmax(kmin, kmax, red);
+  const DigitPlan plan{kmin, 32 - __clz(static_cast<int>(kmax - kmin))};
+  // radix descent from the top: the k-th largest key ut, and how many of the
+  // keys equal to ut are taken (rem)
+  uint32_t rem = static_cast<uint32_t>(k), prefix = 0;
+  for (int l = 0; l < plan.levels(); ++l) {
+    for (int i = threadIdx.x; i < SEL_COPIES * RD_BINS; i += BS_THREADS) hcnt[i] = 0;
+    __syncthreads();
+    for_each_score(sc, L, [&](int j, float x) {
+      const int dg = plan.digit(select_key(x, j, first_forced, bad), l, prefix);
+      if (dg >= 0) atomicAdd(&hcnt[copy * RD_BINS + dg], 1u);
+    });
+    __syncthreads();
+    // thread t owns bins B-1-2t and B-2-2t (descending key order)
+    uint32_t c2[2] = {0, 0};
+#pragma unroll
+    for (int e = 0; e < 2; ++e)
+#pragma unroll
+      for (int c = 0; c < SEL_COPIES; ++c) c2[e] += hcnt[c * RD_BINS + RD_BINS - 1 - 2 * threadIdx.x - e];
+    uint32_t tot;
+    const uint32_t ex = block_exclusive_scan<uint32_t>(c2[0] + c2[1], red, tot);
+    // the one bin where the running count from the top reaches rem
+    if (ex < rem && rem <= ex + c2[0]) {
+      s_chosen = RD_BINS - 1 - 2 * threadIdx.x;
+      s_rem = rem - ex;
+    } else if (ex + c2[0] < rem && rem <= ex + c2[0] + c2[1]) {
+      s_chosen = RD_BINS - 2 - 2 * threadIdx.x;
+      s_rem = rem - ex - c2[0];
+    }
+    __syncthreads();
+    rem = s_rem;
+    prefix = (prefix << (plan.hi(l) - plan.lo(l))) | s_chosen;
+    __syncthreads();
+  }
+  const uint32_t ut = kmin + prefix;
+  const uint32_t need = rem;  // keys equal to ut to take, 1..count(ut)
+
+  // compaction in index order: warp w walks its contiguous segment 32
+  // tokens at a time (coalesced); pass A counts, pass B writes
+  const int seg = (L + BS_WARPS - 1) / BS_WARPS;
+  const int j0 = min(L, warp * seg), j1 = min(L, j0 + seg);
+  // keys of the warp's segment, BS_BATCH steps of 32 loaded at a time
+  auto seg_keys = [&](int jb, uint32_t (&u)[BS_BATCH]) {
+    float v[BS_BATCH];
+#pragma unroll
+    for (int t = 0; t < BS_BATCH; ++t) {
+      const int j = jb + t * 32 + lane;
+      v[t] = j < j1 ? __ldg(sc + j) : 0.f;
+    }
+#pragma unroll
+    for (int t = 0; t < BS_BATCH; ++t) u[t] = select_key(v[t], jb + t * 32 + lane, first_forced, bad);
+  };
+  uint32_t gt = 0, eq = 0;
+  for (int jb = j0; jb < j1; jb += 32 * BS_BATCH) {
+    uint32_t u[BS_BATCH];
+    seg_keys(jb, u);
+#pragma unroll
+    for (int t = 0; t < BS_BATCH; ++t) {
+      const bool in = jb + t * 32 + lane < j1;
+      gt += __popc(__ballot_sync(0xffffffffu, in && u[t] > ut));
+      eq += __popc(__ballot_sync(0xffffffffu, in && u[t] == ut));
+    }
+  }
+  if (lane == 0) {
+    w_gt[warp] = gt;
+    w_eq[warp] = eq;
   }
   __syncthreads();
-  // radix descent from the top: the k-th largest key u_t, and how many of
-  // the keys equal to u_t are taken (s_rem)
-  for (int level = 0; level < 4; ++level) {
-    const int shift = 24 - 8 * level;
-    for (int i = threadIdx.x; i < BS_WARPS * 256; i += BS_THREADS) hcnt[i] = 0;
-    __syncthreads();
-    const uint32_t prefix = s_prefix, mask = s_mask;
-    for (int j = threadIdx.x; j < L; j += BS_THREADS) {
-      const uint32_t u = select_key(sc[j], j, first_forced, bad);
-      if ((u & mask) == prefix) atomicAdd(&hcnt[warp * 256 + ((u >> shift) & 255u)], 1u);
+  if (warp == 0) {   // per-warp bases: ties go to the earlier warps first
+    const uint32_t e = w_eq[lane], g = w_gt[lane];
+    uint32_t ei = e;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, ei, o);
+      if (lane >= o) ei += y;
     }
-    __syncthreads();
-    if (threadIdx.x < 256) {
-      uint32_t c = 0;
-      for (int w = 0; w < BS_WARPS; ++w) c += hcnt[w * 256 + threadIdx.x];
-      hcnt[threadIdx.x] = c;
+    const uint32_t eb = ei - e;                       // ties in earlier warps
+    const uint32_t te = need > eb ? min(e, need - eb) : 0u;
+    const uint32_t t = g + te;
+    uint32_t ti = t;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(0xffffffffu, ti, o);
+      if (lane >= o) ti += y;
     }
-    __syncthreads();
-    if (threadIdx.x == 0) {
-      uint32_t rem = s_rem;
-      int chosen = 0;
-      for (int dgt = 255; dgt >= 0; --dgt) {
-        if (hcnt[dgt] < rem) {
-          rem -= hcnt[dgt];
-        } else {
-          chosen = dgt;
-          break;
-        }
-      }
-      s_rem = rem;
-      s_prefix = prefix | (static_cast<uint32_t>(chosen) << shift);
-      s_mask = mask | (255u << shift);
-    }
-    __syncthreads();
+    w_base[lane] = ti - t;
+    w_eqb[lane] = eb;
   }
-  const uint32_t ut = s_prefix;
-  const uint32_t need = s_rem;  // keys equal to ut to take, 1..count(ut)
-
-  // compaction in index order: thread t owns the contiguous range [j0, j1)
-  const int per = (L + BS_THREADS - 1) / BS_THREADS;
-  const int j0 = min(L, static_cast<int>(threadIdx.x) * per);
-  const int j1 = min(L, j0 + per);
-  uint32_t gt = 0, eq = 0;
-  for (int j = j0; j < j1; ++j) {
-    const uint32_t u = select_key(sc[j], j, first_forced, bad);
-    gt += (u > ut);
-    eq += (u == ut);
-  }
-  uint32_t eq_total;
-  const uint32_t eq_before = block_exclusive_scan(eq, red, eq_total);
-  const uint32_t take_eq = need > eq_before ? min(eq, need - eq_before) : 0u;
-  uint32_t cnt_total;
-  uint32_t pos = block_exclusive_scan(gt + take_eq, red, cnt_total);
-  uint32_t eq_seen = eq_before;
-  for (int j = j0; j < j1; ++j) {
-    const uint32_t u = select_key(sc[j], j, first_forced, bad);
-    bool take = u > ut;
-    if (u == ut) {
-      take = eq_seen < need;
-      ++eq_seen;
+  __syncthreads();
+  uint32_t pos = w_base[warp], eq_seen = w_eqb[warp];
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int jb = j0; jb < j1; jb += 32 * BS_BATCH) {
+    uint32_t u[BS_BATCH];
+    seg_keys(jb, u);
+#pragma unroll
+    for (int t = 0; t < BS_BATCH; ++t) {
+      const int j = jb + t * 32 + lane;
+      const bool is_eq = j < j1 && u[t] == ut;
+      const uint32_t eqm = __ballot_sync(0xffffffffu, is_eq);
+      const bool take = j < j1 && (u[t] > ut || (is_eq && eq_seen + __popc(eqm & lt) < need));
+      const uint32_t tm = __ballot_sync(0xffffffffu, take);
+      if (take) out[pos + __popc(tm & lt)] = j;
+      pos += __popc(tm);
+      eq_seen += __popc(eqm);
     }
-    if (take) out[pos++] = j;
   }
   for (int i = k + threadIdx.x; i < cap; i += BS_THREADS) out[i] = -1;
 }

@@ -315,6 +315,37 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
   asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
   return d;
 }
+// 2^x for a pair of fp32 values on the FMA and integer pipes, without the
+// MUFU unit (which issues one ex2 per 8 clocks per SMSP on sm_100a, as many
+// exponentials per clock as the tensor core consumes at d = 128: doing part
+// of them here gives the softmax slack).  Cody and Waite's range reduction
+// x = n + r with n = rint(x) and |r| <= 1/2 (n taken from the low mantissa
+// bits of x + 1.5 * 2^23), then a cubic for 2^r -- a minimax fit of the
+// relative error on [-1/2, 1/2] made for this library, maximum 7.5e-5 --
+// scaled by 2^n through the exponent field.  x is first raised to -125 so
+// the scaled exponent stays normal (2^-125, about 2e-38, stands in for
+// zero); callers keep x <= 127.
+__device__ __forceinline__ void exp2_poly_x2(uint64_t x, float& y0, float& y1) {
+  float a, b;
+  f2_unpack(x, a, b);
+  a = fmaxf(a, -125.f);
+  b = fmaxf(b, -125.f);
+  const uint64_t xc = f2_pack(a, b);
+  const uint64_t t = f2_add(xc, f2_pack(12582912.f, 12582912.f));         // 1.5 * 2^23 + rint(x)
+  const uint64_t n = f2_add(t, f2_pack(-12582912.f, -12582912.f));        // rint(x)
+  const uint64_t r = f2_fma(n, f2_pack(-1.f, -1.f), xc);                  // x - rint(x)
+  uint64_t q = f2_fma(f2_pack(0.05517166905792616f, 0.05517166905792616f), r,
+                      f2_pack(0.2426111221932161f, 0.2426111221932161f));
+  q = f2_fma(q, r, f2_pack(0.6932609854606553f, 0.6932609854606553f));
+  q = f2_fma(q, r, f2_pack(0.9999280735394012f, 0.9999280735394012f));
+  float q0, q1, t0, t1;
+  f2_unpack(q, q0, q1);
+  f2_unpack(t, t0, t1);
+  // the low bits of t hold n; shifted by 23 they land in the exponent field
+  y0 = __uint_as_float(__float_as_uint(q0) + (__float_as_uint(t0) << 23));
+  y1 = __uint_as_float(__float_as_uint(q1) + (__float_as_uint(t1) << 23));
+}
+
 // Three-input maximum.
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float d;

@@ -10,6 +10,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdint>
@@ -31,21 +32,33 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-// Key tiles per score CTA: long enough spans that the grid is a few waves of
-// 148 SMs (per-CTA set-up then amortises), never below 16 tiles.
-int score_chunk_tiles(const tsa_params* p) {
+// Proxy-score work split (see score.cuh): each head's window padded to a
+// multiple of 32 rows, as many query heads of a KV group per CTA as fit in
+// 512 packed rows, and key chunks sized so the grid is about two waves of
+// 148 SMs (one CTA per SM), never below 4 key tiles.
+struct ScorePlan {
+  int W32, GH, n_hg, n_rp, MT, chunk_tiles, n_chunks;
+};
+
+ScorePlan score_plan(const tsa_params* p) {
+  ScorePlan s;
+  const int G = p->Hq / p->Hkv;
+  s.W32 = (p->w + 31) / 32 * 32;
+  s.GH = s.W32 <= tsa::SC_PASS_ROWS ? std::min(G, tsa::SC_PASS_ROWS / s.W32) : 1;
+  s.n_hg = (G + s.GH - 1) / s.GH;
+  const int rows = s.GH * s.W32;
+  s.n_rp = (rows + tsa::SC_PASS_ROWS - 1) / tsa::SC_PASS_ROWS;
+  s.MT = s.n_rp > 1 ? tsa::SC_MAX_MT : (rows + 127) / 128;
   const int tiles = (p->L + tsa::SC_KEYS - 1) / tsa::SC_KEYS;
-  const int heads = p->B * p->Hq;
-  int per_head = (148 * 4) / heads;
-  per_head = per_head < 1 ? 1 : per_head;
-  const int ct = (tiles + per_head - 1) / per_head;
-  return ct < tsa::SC_MIN_CHUNK_TILES ? tsa::SC_MIN_CHUNK_TILES : ct;
+  const int ctas = p->B * p->Hkv * s.n_hg;
+  const int per = std::max(1, (2 * 148) / ctas);
+  s.chunk_tiles = std::max(tsa::SC_MIN_CHUNK_TILES, (tiles + per - 1) / per);
+  const int span = s.chunk_tiles * tsa::SC_KEYS;
+  s.n_chunks = (p->L + span - 1) / span;
+  return s;
 }
 
-int score_chunks(const tsa_params* p) {
-  const int span = score_chunk_tiles(p) * tsa::SC_KEYS;
-  return (p->L + span - 1) / span;
-}
+int score_chunks(const tsa_params* p) { return score_plan(p).n_chunks; }
 
 // Workspace layout.  Stage part: status word (+ abort words), score scratch,
 // per-head budget scratch.
@@ -195,8 +208,8 @@ std::atomic<int> g_attn64[kMaxDevices], g_attn128[kMaxDevices], g_gath64[kMaxDev
     g_select[kMaxDevices], g_blk64[kMaxDevices], g_blk128[kMaxDevices], g_blks64[kMaxDevices],
     g_blks128[kMaxDevices];
 
-constexpr int kBudgetSmem = tsa::BS_WARPS * 256 * (8 + 4);
-constexpr int kSelectSmem = tsa::BS_WARPS * 256 * 4;
+constexpr int kBudgetSmem = tsa::BUD_SMEM;
+constexpr int kSelectSmem = tsa::SEL_SMEM;
 
 // ---------------------------------------------------------------- launchers
 // Tensor map over the caller's q, k or v (`heads` heads): per-sequence
@@ -210,10 +223,10 @@ bool make_caller_map(CUtensorMap* m, const tsa_params* p, const void* base, int 
 tsa_status run_score(const tsa_params* p, const void* q, const void* k, float* scores, void* ws,
                      cudaStream_t st) {
   const WsLayout w = layout_of(p);
-  const int bhq = p->B * p->Hq;
+  const ScorePlan sp = score_plan(p);
   CUtensorMap mq, mk;
   const bool tm = token_major(p);
-  if (!make_caller_map(&mq, p, q, p->Hq, tsa::SC_ROWS) || !make_caller_map(&mk, p, k, p->Hkv, tsa::SC_KEYS))
+  if (!make_caller_map(&mq, p, q, p->Hq, tsa::SC_QBOX) || !make_caller_map(&mk, p, k, p->Hkv, tsa::SC_KEYS))
     return TSA_ERR_CUDA;
   tsa::ScoreArgs a;
   a.scores = scores;
@@ -227,16 +240,20 @@ tsa_status run_score(const tsa_params* p, const void* q, const void* k, float* s
   a.Hq = p->Hq;
   a.Hkv = p->Hkv;
   a.G = p->Hq / p->Hkv;
-  a.n_chunks = score_chunks(p);
-  a.chunk_tiles = score_chunk_tiles(p);
-  a.n_rb = (p->w + tsa::SC_ROWS - 1) / tsa::SC_ROWS;
+  a.W32 = sp.W32;
+  a.GH = sp.GH;
+  a.n_hg = sp.n_hg;
+  a.n_rp = sp.n_rp;
+  a.MT = sp.MT;
+  a.n_chunks = sp.n_chunks;
+  a.chunk_tiles = sp.chunk_tiles;
   a.scale_log2 = scale_of(p) * 1.4426950408889634f;
   a.limit_ns = limit_ns_of(p);
   a.token_major = tm ? 1 : 0;
   a.test_stall = (p->flags & TSA_FLAG_TEST_STALL_SCORE) ? 1 : 0;
   a.seqs = seqs_of(p);
-  const dim3 grid(a.n_chunks, bhq);
-  const int rows = bhq * p->w;
+  const dim3 grid(sp.n_chunks, p->B * p->Hkv * sp.n_hg);
+  const int rows = p->B * p->Hq * p->w;
   if (cudaMemsetAsync(a.abort_word, 0, sizeof(uint32_t), st) != cudaSuccess) return TSA_ERR_CUDA;
   if (p->d == 128) {
     constexpr int sm = tsa::ScoreLayout<128>::ALLOC;
@@ -281,12 +298,6 @@ tsa_status run_select(const tsa_params* p, const float* scores, const int32_t* k
   return launch_ok();
 }
 
-int copy_grid(long long rows, int lanes_per_row) {
-  long long blocks = (rows * lanes_per_row + 255) / 256;
-  const long long cap = 148LL * 8;
-  return static_cast<int>(blocks < cap ? (blocks < 1 ? 1 : blocks) : cap);
-}
-
 tsa_status run_gather(const tsa_params* p, const void* q, const void* k, const void* v, const int32_t* idx,
                       const int32_t* k_seq, void* qc, void* kc, void* vc, uint32_t* status, cudaStream_t st) {
   tsa::GatherArgs a;
@@ -302,15 +313,18 @@ tsa_status run_gather(const tsa_params* p, const void* q, const void* k, const v
   a.kc = static_cast<__nv_bfloat16*>(kc);
   a.vc = static_cast<__nv_bfloat16*>(vc);
   a.status = status;
+  a.B = p->B;
   a.L = p->L;
   a.Hq = p->Hq;
   a.Hkv = p->Hkv;
   a.G = p->Hq / p->Hkv;
-  a.total_rows = static_cast<long long>(p->B) * p->Hq * p->L;
+  // one resident wave of 4 CTAs per SM, each walking work items
+  const long long items = static_cast<long long>(p->B) * p->Hkv * ((p->L + tsa::GT_ROWS - 1) / tsa::GT_ROWS);
+  const int grid = static_cast<int>(items < 148LL * 4 ? items : 148LL * 4);
   if (p->d == 128)
-    tsa::gather_kernel<128><<<copy_grid(a.total_rows, 16), 256, 0, st>>>(a);
+    tsa::gather_kernel<128><<<grid, 256, 0, st>>>(a);
   else
-    tsa::gather_kernel<64><<<copy_grid(a.total_rows, 8), 256, 0, st>>>(a);
+    tsa::gather_kernel<64><<<grid, 256, 0, st>>>(a);
   return launch_ok();
 }
 
