@@ -47,7 +47,7 @@ KERNELS_PER_FORWARD = 9  # score x3, budget, budget finalize, select, gather, at
 ATTN_DRAM_BYTES_PER_KEPT_ROW = None
 ATTN_TRAFFIC_NOTE = "not yet captured for the current kernel"
 SMS = 148
-EX2_PER_CLK_SM = 32
+EX2_PER_CLK_SM = 16   # ex2.approx on B200, measured: one warp instruction per 8 clocks per SMSP
 
 
 def stage_algorithmic_bytes(wl, kept_np, idx) -> dict:
@@ -688,7 +688,7 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
     stage_roof["score"]["exp_per_s"] = exps / (stage_ms["score"] * 1e-3)
     stage_roof["score"]["exp_frac"] = stage_roof["score"]["exp_per_s"] / ex2_peak
     stage_roof["score"]["exp_peak_note"] = (f"{EX2_PER_CLK_SM} ex2/clk/SM x {SMS} SMs x the median sampled SM clock "
-                                            "(ex2.approx rate of one warp instruction per 4 clocks per SMSP)")
+                                            "(ex2.approx: one warp instruction per 8 clocks per SMSP, measured)")
 
     job_flops = dense_flops(wl_all) * (1 if sharded else world)   # the work of all ranks together
     value = job_value(wl_all, world, ms, sharded)

@@ -286,20 +286,24 @@ __global__ void __launch_bounds__(SC_THREADS, 1)
     float* red = reinterpret_cast<float*>(gbase + C::OFF_RED);
     bool live = true;
     for (int rp = 0; live && rp < n_rp; ++rp) {
-      // this thread's packed row in M tile m: rp*512 + m*128 + 32*lq + lane
+      // this thread's packed row in M tile m: rp*512 + m*128 + 32*lq + lane;
+      // its head, position (or -1: padding or outside the window) and, in
+      // the second pass, its (max, 1/sum) statistics
       float m_run[SC_MAX_MT];
       double z_run[SC_MAX_MT];
       float2 st_row[SC_MAX_MT];
+      int pos_m[SC_MAX_MT];
 #pragma unroll
       for (int m = 0; m < SC_MAX_MT; ++m) {
         m_run[m] = -INFINITY;
         z_run[m] = 0.0;
         st_row[m] = make_float2(0.f, 0.f);
+        const int gr = rp * SC_PASS_ROWS + m * 128 + lq * 32 + lane;
+        const int hl = gr / a.W32, wr = gr - hl * a.W32;
+        const bool row_ok = m < MT && gr < R && wr < wb;
+        pos_m[m] = row_ok ? pos0 + wr : -1;
         if constexpr (kPass2) {
-          const int gr = rp * SC_PASS_ROWS + m * 128 + lq * 32 + lane;
-          const int hl = gr / a.W32, wr = gr - hl * a.W32;
-          if (m < MT && gr < R && wr < wb)
-            st_row[m] = a.stats[(static_cast<size_t>(b) * a.Hq + h0 + hl) * a.w + wr];
+          if (row_ok) st_row[m] = a.stats[(static_cast<size_t>(b) * a.Hq + h0 + hl) * a.w + wr];
         }
       }
       for (int kt = 0; live && kt < n_kt; ++kt) {
@@ -318,18 +322,35 @@ __global__ void __launch_bounds__(SC_THREADS, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(bar(SB_SFREE + m));
-          const int gr = rp * SC_PASS_ROWS + m * 128 + lq * 32 + lane;
-          const int hl = gr / a.W32, wr = gr - hl * a.W32;
-          const bool row_ok = gr < R && wr < wb;
-          const int pos = pos0 + wr;
+          // logits: the two partial accumulators summed (packed pairs)
+          uint64_t xs[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) xs[e] = f2_add(f2_pack(x[2 * e], x[2 * e + 1]), f2_pack(xb[2 * e], xb[2 * e + 1]));
+          // every key of this thread's 16 is visible to its row (the common
+          // case), or some are masked: past the row's position (causal) or
+          // past the sequence (this only happens near the window)
+          const int pos = pos_m[m];
+          const bool full = kbase + 15 <= pos && kbase + 15 < Lb;
+          if (!full) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              float v0, v1;
+              f2_unpack(xs[e], v0, v1);
+              const int k0 = kbase + 2 * e;
+              v0 = (k0 <= pos && k0 < Lb) ? v0 : -INFINITY;
+              v1 = (k0 + 1 <= pos && k0 + 1 < Lb) ? v1 : -INFINITY;
+              xs[e] = f2_pack(v0, v1);
+            }
+          }
           if constexpr (!kPass2) {
             float mx = -INFINITY;
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int key = kbase + e;
-              x[e] = (row_ok && key <= pos && key < Lb) ? (x[e] + xb[e]) * sl2 : -INFINITY;
-              mx = fmaxf(mx, x[e]);
+            for (int e = 0; e < 8; ++e) {
+              float v0, v1;
+              f2_unpack(xs[e], v0, v1);
+              mx = fmax3(mx, v0, v1);
             }
+            mx *= sl2;                                       // sl2 > 0: the max of the scaled logits
             if (mx != -INFINITY) {
               // lazy reference: keep m_run unless this tile's max passes it
               // by more than 2^8 (terms up to 256 are summed safely in fp32)
@@ -337,20 +358,31 @@ __global__ void __launch_bounds__(SC_THREADS, 1)
                 if (m_run[m] != -INFINITY) z_run[m] *= exp2(static_cast<double>(m_run[m]) - mx);
                 m_run[m] = mx;
               }
-              const float ref = m_run[m];
-              float z4[4] = {0.f, 0.f, 0.f, 0.f};
+              const uint64_t sl2x2 = f2_pack(sl2, sl2), nref = f2_pack(-m_run[m], -m_run[m]);
+              uint64_t z2[2] = {0ull, 0ull};
 #pragma unroll
-              for (int e = 0; e < 16; ++e) z4[e & 3] += ex2_approx(x[e] - ref);
-              z_run[m] += static_cast<double>((z4[0] + z4[1]) + (z4[2] + z4[3]));
+              for (int e = 0; e < 8; ++e) {
+                float v0, v1;
+                f2_unpack(f2_fma(xs[e], sl2x2, nref), v0, v1);
+                z2[e & 1] = f2_add(z2[e & 1], f2_pack(ex2_approx(v0), ex2_approx(v1)));
+              }
+              float za, zb2, zc, zd;
+              f2_unpack(z2[0], za, zb2);
+              f2_unpack(z2[1], zc, zd);
+              z_run[m] += static_cast<double>((za + zb2) + (zc + zd));
             }
           } else {
             const float2 sr = st_row[m];
+            const uint64_t sl2x2 = f2_pack(sl2, sl2), nm = f2_pack(-sr.x, -sr.x), iz = f2_pack(sr.y, sr.y);
+            float pv[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int key = kbase + e;
-              x[e] = (row_ok && key <= pos && key < Lb) ? ex2_approx(fmaf(x[e] + xb[e], sl2, -sr.x)) * sr.y : 0.f;
+            for (int e = 0; e < 8; ++e) {
+              float v0, v1;
+              f2_unpack(f2_fma(xs[e], sl2x2, nm), v0, v1);
+              // a masked logit is -inf, and ex2 of -inf is +0
+              f2_unpack(f2_mul(f2_pack(ex2_approx(v0), ex2_approx(v1)), iz), pv[2 * e], pv[2 * e + 1]);
             }
-            const float cs = warp_column_sums16(x, lane);
+            const float cs = warp_column_sums16(pv, lane);
             if (lane < 16) red[((n & 1) * SC_MAX_MT * 4 + m * 4 + lq) * SC_KEYS + cg * 16 + lane] = cs;
           }
         }
