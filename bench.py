@@ -41,11 +41,12 @@ UNIT = "TFLOP/s (effective: dense causal attention FLOPs / TSA time)"
 DEFAULT_WORKLOAD = "c4_L128K_gqa"
 KERNELS_PER_FORWARD = 9  # score x3, budget, budget finalize, select, gather, attention, scatter
 # DRAM bytes per kept (head, row) of the forward's attention kernel, from ncu
-# dram__bytes_read.sum + dram__bytes_write.sum of one launch (None until the
-# current kernel has been captured); DRAM traffic grows with kept rows, not
-# with FLOPs (algorithmic: 3 x 256 B read + 256 B written per kept row).
-ATTN_DRAM_BYTES_PER_KEPT_ROW = None
-ATTN_TRAFFIC_NOTE = "not yet captured for the current kernel"
+# dram__bytes_read.sum + dram__bytes_write.sum of one launch; DRAM traffic
+# grows with kept rows, not with FLOPs (algorithmic: 3 x 256 B read + 256 B
+# written per kept row).
+ATTN_DRAM_BYTES_PER_KEPT_ROW = 805.7e6 / (32 * 25147)
+ATTN_TRAFFIC_NOTE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch of the same kernel on the 32K "
+                     "workload (805.7 MB for 32 x 25147 kept rows), scaled by kept rows")
 SMS = 148
 EX2_PER_CLK_SM = 16   # ex2.approx on B200, measured: one warp instruction per 8 clocks per SMSP
 

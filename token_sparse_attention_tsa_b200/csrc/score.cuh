@@ -49,7 +49,7 @@ constexpr int SC_LOAD_WARP = SC_ROW_WARPS + 1;
 constexpr int SC_MAX_MT = 4;             // M tiles (128 packed rows each) per row pass
 constexpr int SC_PASS_ROWS = SC_MAX_MT * 128;
 constexpr int SC_STAGES = 3;
-constexpr int SC_MIN_CHUNK_TILES = 4;    // smallest key span of a CTA, in tiles (256 keys)
+constexpr int SC_MIN_CHUNK_TILES = 16;   // smallest key span of a CTA, in tiles (1024 keys)
 
 struct ScoreArgs {
   float* scores;           // [B*Hq, L]

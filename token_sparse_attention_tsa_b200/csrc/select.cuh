@@ -158,8 +158,16 @@ constexpr int RD_BITS = 11;                 // digit width of the radix descent
 constexpr int RD_BINS = 1 << RD_BITS;       // 2048 bins per level
 constexpr int BUD_COPIES = 4;               // budget histogram copies (eight warps each)
 constexpr int SEL_COPIES = 8;               // select histogram copies (four warps each)
-constexpr int BUD_SMEM = BUD_COPIES * RD_BINS * (8 + 4);
-constexpr int SEL_SMEM = SEL_COPIES * RD_BINS * 4;
+// Each head is one thread-block cluster of BS_CLUSTER CTAs, each taking a
+// contiguous quarter of the keys; a CTA publishes its merged histogram in
+// its shared memory (two buffers, by level parity) and every CTA reads the
+// BS_CLUSTER published histograms in rank order, so all of them take the
+// same, timing-independent decision.
+constexpr int BS_CLUSTER = 4;
+constexpr int BUD_PUB = RD_BINS * (8 + 4);          // one published histogram (sum, count)
+constexpr int BUD_SMEM = BUD_COPIES * RD_BINS * (8 + 4) + 2 * BUD_PUB;
+constexpr int SEL_PUB = RD_BINS * 4;
+constexpr int SEL_SMEM = SEL_COPIES * RD_BINS * 4 + 2 * SEL_PUB;
 
 // Digit plan of a descent over r = key - kmin: nb is the bit length of
 // kmax - kmin; level l covers bits [lo(l), hi(l)) of r, 11 bits at a time
@@ -193,27 +201,34 @@ struct BudgetArgs {
   Seqs seqs;            // sequence lengths L_b
 };
 
-// grid: B*Hq CTAs of 1024 threads; dynamic smem: BUD_SMEM (count and mass
-// histograms, BUD_COPIES copies).
-__global__ void __launch_bounds__(BS_THREADS, 1) budget_kernel(const BudgetArgs a) {
+// grid: B*Hq clusters of BS_CLUSTER CTAs of 1024 threads; dynamic smem:
+// BUD_SMEM (count and mass histograms, BUD_COPIES working copies, two
+// published buffers).
+__global__ void __cluster_dims__(BS_CLUSTER, 1, 1) __launch_bounds__(BS_THREADS, 1)
+    budget_kernel(const BudgetArgs a) {
   extern __shared__ __align__(16) uint8_t bsm[];
   unsigned long long* hsum = reinterpret_cast<unsigned long long*>(bsm);           // [copies][bins]
   uint32_t* hcnt = reinterpret_cast<uint32_t*>(bsm + BUD_COPIES * RD_BINS * 8);    // [copies][bins]
+  uint8_t* pub = bsm + BUD_COPIES * RD_BINS * 12;                                  // [2][sum bins, count bins]
   __shared__ unsigned long long red64[33];
   __shared__ uint32_t red32[64];
-  __shared__ unsigned long long s_rem;
-  __shared__ uint32_t s_below, s_chosen;
+  __shared__ unsigned long long s_rem, s_stat_tot;
+  __shared__ uint32_t s_below, s_chosen, s_stat_min, s_stat_max;
 
-  const int bh = blockIdx.x;
+  const uint32_t crank = cluster_rank();
+  const int bh = blockIdx.x / BS_CLUSTER;
   const float* sc = a.scores + static_cast<size_t>(bh) * a.L;
   const int copy = (threadIdx.x >> 5) % BUD_COPIES;
   bool bad = false, bad_seq = false;
   const int Lb = a.seqs.len_ok(bh / a.Hq, bad_seq);
+  const int span = (Lb + BS_CLUSTER - 1) / BS_CLUSTER;
+  const int j0 = min(Lb, static_cast<int>(crank) * span), n = min(Lb, j0 + span) - j0;
+  const float* scc = sc + j0;                       // this CTA's keys [j0, j0 + n)
 
-  // pass 0: total mass and the key range
+  // pass 0: total mass and the key range (this CTA's part, then the cluster's)
   unsigned long long tot = 0;
   uint32_t kmin = 0xffffffffu, kmax = 0u;
-  for_each_score(sc, Lb, [&](int, float x) {
+  for_each_score(scc, n, [&](int, float x) {
     const uint32_t u = score_key(x, bad);
     tot += mass_of_key(u);
     kmin = min(kmin, u);
@@ -221,6 +236,29 @@ __global__ void __launch_bounds__(BS_THREADS, 1) budget_kernel(const BudgetArgs 
   });
   tot = block_sum<unsigned long long>(tot, red64);
   block_minmax(kmin, kmax, red32);
+  if (threadIdx.x == 0) {
+    s_stat_tot = tot;
+    s_stat_min = kmin;
+    s_stat_max = kmax;
+  }
+  cluster_sync();
+  if (threadIdx.x == 0) {
+    unsigned long long t = 0;
+    uint32_t mn = 0xffffffffu, mx = 0u;
+    for (uint32_t rk = 0; rk < BS_CLUSTER; ++rk) {
+      t += ld_cluster_u64(cluster_map(smem_u32(&s_stat_tot), rk));
+      mn = min(mn, ld_cluster_u32(cluster_map(smem_u32(&s_stat_min), rk)));
+      mx = max(mx, ld_cluster_u32(cluster_map(smem_u32(&s_stat_max), rk)));
+    }
+    red64[0] = t;
+    red32[0] = mn;
+    red32[1] = mx;
+  }
+  __syncthreads();
+  tot = red64[0];
+  kmin = red32[0];
+  kmax = red32[1];
+  __syncthreads();
   const unsigned long long T =
       static_cast<unsigned long long>(floor(__dmul_rn(a.tau, __ull2double_rn(tot))));
   const DigitPlan plan{kmin, Lb > 0 ? 32 - __clz(static_cast<int>(kmax - kmin)) : 0};
@@ -233,7 +271,7 @@ __global__ void __launch_bounds__(BS_THREADS, 1) budget_kernel(const BudgetArgs 
       hcnt[i] = 0;
     }
     __syncthreads();
-    for_each_score(sc, Lb, [&](int, float x) {
+    for_each_score(scc, n, [&](int, float x) {
       const uint32_t u = score_key(x, bad);
       const int dg = plan.digit(u, l, prefix);
       if (dg >= 0) {
@@ -242,15 +280,32 @@ __global__ void __launch_bounds__(BS_THREADS, 1) budget_kernel(const BudgetArgs 
       }
     });
     __syncthreads();
-    // thread t owns bins 2t and 2t+1 (ascending key order)
-    unsigned long long s2[2] = {0, 0}, c2[2] = {0, 0};
-#pragma unroll
-    for (int e = 0; e < 2; ++e)
+    // publish this CTA's histogram (its copies merged) in buffer l & 1
+    unsigned long long* ps = reinterpret_cast<unsigned long long*>(pub + (l & 1) * BUD_PUB);
+    uint32_t* pc = reinterpret_cast<uint32_t*>(pub + (l & 1) * BUD_PUB + RD_BINS * 8);
+    for (int i = threadIdx.x; i < RD_BINS; i += BS_THREADS) {
+      unsigned long long sv = 0;
+      uint32_t cv = 0;
 #pragma unroll
       for (int c = 0; c < BUD_COPIES; ++c) {
-        s2[e] += hsum[c * RD_BINS + 2 * threadIdx.x + e];
-        c2[e] += hcnt[c * RD_BINS + 2 * threadIdx.x + e];
+        sv += hsum[c * RD_BINS + i];
+        cv += hcnt[c * RD_BINS + i];
       }
+      ps[i] = sv;
+      pc[i] = cv;
+    }
+    cluster_sync();
+    // thread t owns bins 2t and 2t+1 (ascending key order): the cluster's
+    // totals, summed over the CTAs in rank order
+    unsigned long long s2[2] = {0, 0}, c2[2] = {0, 0};
+    for (uint32_t rk = 0; rk < BS_CLUSTER; ++rk) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int bin = 2 * threadIdx.x + e;
+        s2[e] += ld_cluster_u64(cluster_map(smem_u32(ps + bin), rk));
+        c2[e] += ld_cluster_u32(cluster_map(smem_u32(pc + bin), rk));
+      }
+    }
     unsigned long long tot_s, tot_c;
     const unsigned long long es = block_exclusive_scan<unsigned long long>(s2[0] + s2[1], red64, tot_s);
     const unsigned long long ec = block_exclusive_scan<unsigned long long>(c2[0] + c2[1], red64, tot_c);
@@ -276,7 +331,7 @@ __global__ void __launch_bounds__(BS_THREADS, 1) budget_kernel(const BudgetArgs 
     prefix = (prefix << (plan.hi(l) - plan.lo(l))) | s_chosen;
     __syncthreads();
   }
-  if (threadIdx.x == 0) {
+  if (threadIdx.x == 0 && crank == 0) {
     uint32_t p = below;
     if (!done) {  // the descent ended on one key value: its tokens share one mass
       const unsigned long long qstar = mass_of_key(kmin + prefix);   // > 0 here
@@ -288,6 +343,7 @@ __global__ void __launch_bounds__(BS_THREADS, 1) budget_kernel(const BudgetArgs 
     if (bad_seq && a.status) atomicOr(a.status, 0x4u);
   }
   if (a.status && __syncthreads_or(bad) && threadIdx.x == 0) atomicOr(a.status, 0x1u);
+  cluster_sync();   // no CTA leaves while another may still read its shared memory
 }
 
 // k_seq[b] from the heads' counts: mode 1 the ceiling of their mean, mode 2
@@ -341,16 +397,20 @@ __device__ __forceinline__ uint32_t select_key(float s, int j, int first_forced,
   return j >= first_forced ? 0xffffffffu : u;
 }
 
-// grid: B*Hq CTAs of 1024 threads; dynamic smem: SEL_SMEM (count
-// histograms, SEL_COPIES copies).
-__global__ void __launch_bounds__(BS_THREADS, 1) select_kernel(const SelectArgs a) {
+// grid: B*Hq clusters of BS_CLUSTER CTAs of 1024 threads; dynamic smem:
+// SEL_SMEM (count histograms, SEL_COPIES working copies, two published
+// buffers).
+__global__ void __cluster_dims__(BS_CLUSTER, 1, 1) __launch_bounds__(BS_THREADS, 1)
+    select_kernel(const SelectArgs a) {
   extern __shared__ __align__(16) uint8_t ssm[];
-  uint32_t* hcnt = reinterpret_cast<uint32_t*>(ssm);  // [copies][bins]
+  uint32_t* hcnt = reinterpret_cast<uint32_t*>(ssm);                     // [copies][bins]
+  uint32_t* pub = reinterpret_cast<uint32_t*>(ssm + SEL_COPIES * RD_BINS * 4);   // [2][bins]
   __shared__ uint32_t red[64];
-  __shared__ uint32_t s_rem, s_chosen;
+  __shared__ uint32_t s_rem, s_chosen, s_min, s_max, s_gt, s_eq;
   __shared__ uint32_t w_gt[BS_WARPS], w_eq[BS_WARPS], w_base[BS_WARPS], w_eqb[BS_WARPS];
 
-  const int bh = blockIdx.x;
+  const uint32_t crank = cluster_rank();
+  const int bh = blockIdx.x / BS_CLUSTER;
   const int cap = a.L;                               // row capacity of idx
   const int L = a.seqs.len(bh / a.Hq);               // this sequence's length
   const float* sc = a.scores + static_cast<size_t>(bh) * cap;
@@ -359,24 +419,44 @@ __global__ void __launch_bounds__(BS_THREADS, 1) select_kernel(const SelectArgs 
   const int first_forced = L - (a.keep_recent < L ? a.keep_recent : L);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int copy = warp % SEL_COPIES;
+  // this CTA's keys [c0, c0 + n) and its share of the index row
+  const int span = (L + BS_CLUSTER - 1) / BS_CLUSTER;
+  const int c0 = min(L, static_cast<int>(crank) * span), n = min(L, c0 + span) - c0;
+  const int cspan = (cap + BS_CLUSTER - 1) / BS_CLUSTER;
+  const int o0 = min(cap, static_cast<int>(crank) * cspan), o1 = min(cap, o0 + cspan);
   bool bad = false;
 
-  if (k == L) {  // everything kept
-    for (int i = threadIdx.x; i < cap; i += BS_THREADS) out[i] = i < L ? i : -1;
+  if (k == L || k == 0) {  // everything kept, or nothing (the same for the whole cluster)
+    for (int i = o0 + threadIdx.x; i < o1; i += BS_THREADS) out[i] = (k == L && i < L) ? i : -1;
     return;
   }
-  if (k == 0) {
-    for (int i = threadIdx.x; i < cap; i += BS_THREADS) out[i] = -1;
-    return;
-  }
-  // pass 0: the key range
+  auto key_at = [&](int j, float x) { return select_key(x, j, first_forced, bad); };
+  // pass 0: the key range (this CTA's part, then the cluster's)
   uint32_t kmin = 0xffffffffu, kmax = 0u;
-  for_each_score(sc, L, [&](int j, float x) {
-    const uint32_t u = select_key(x, j, first_forced, bad);
+  for_each_score(sc + c0, n, [&](int jl, float x) {
+    const uint32_t u = key_at(c0 + jl, x);
     kmin = min(kmin, u);
     kmax = max(kmax, u);
   });
   block_minmax(kmin, kmax, red);
+  if (threadIdx.x == 0) {
+    s_min = kmin;
+    s_max = kmax;
+  }
+  cluster_sync();
+  if (threadIdx.x == 0) {
+    uint32_t mn = 0xffffffffu, mx = 0u;
+    for (uint32_t rk = 0; rk < BS_CLUSTER; ++rk) {
+      mn = min(mn, ld_cluster_u32(cluster_map(smem_u32(&s_min), rk)));
+      mx = max(mx, ld_cluster_u32(cluster_map(smem_u32(&s_max), rk)));
+    }
+    red[0] = mn;
+    red[1] = mx;
+  }
+  __syncthreads();
+  kmin = red[0];
+  kmax = red[1];
+  __syncthreads();
   const DigitPlan plan{kmin, 32 - __clz(static_cast<int>(kmax - kmin))};
   // radix descent from the top: the k-th largest key ut, and how many of the
   // keys equal to ut are taken (rem)
@@ -384,17 +464,27 @@ __global__ void __launch_bounds__(BS_THREADS, 1) select_kernel(const SelectArgs 
   for (int l = 0; l < plan.levels(); ++l) {
     for (int i = threadIdx.x; i < SEL_COPIES * RD_BINS; i += BS_THREADS) hcnt[i] = 0;
     __syncthreads();
-    for_each_score(sc, L, [&](int j, float x) {
-      const int dg = plan.digit(select_key(x, j, first_forced, bad), l, prefix);
+    for_each_score(sc + c0, n, [&](int jl, float x) {
+      const int dg = plan.digit(key_at(c0 + jl, x), l, prefix);
       if (dg >= 0) atomicAdd(&hcnt[copy * RD_BINS + dg], 1u);
     });
     __syncthreads();
-    // thread t owns bins B-1-2t and B-2-2t (descending key order)
+    uint32_t* pb = pub + (l & 1) * RD_BINS;          // publish the merged copies
+    for (int i = threadIdx.x; i < RD_BINS; i += BS_THREADS) {
+      uint32_t cv = 0;
+#pragma unroll
+      for (int c = 0; c < SEL_COPIES; ++c) cv += hcnt[c * RD_BINS + i];
+      pb[i] = cv;
+    }
+    cluster_sync();
+    // thread t owns bins B-1-2t and B-2-2t (descending key order): the
+    // cluster's counts, summed over the CTAs in rank order
     uint32_t c2[2] = {0, 0};
+    for (uint32_t rk = 0; rk < BS_CLUSTER; ++rk) {
 #pragma unroll
-    for (int e = 0; e < 2; ++e)
-#pragma unroll
-      for (int c = 0; c < SEL_COPIES; ++c) c2[e] += hcnt[c * RD_BINS + RD_BINS - 1 - 2 * threadIdx.x - e];
+      for (int e = 0; e < 2; ++e)
+        c2[e] += ld_cluster_u32(cluster_map(smem_u32(pb + RD_BINS - 1 - 2 * threadIdx.x - e), rk));
+    }
     uint32_t tot;
     const uint32_t ex = block_exclusive_scan<uint32_t>(c2[0] + c2[1], red, tot);
     // the one bin where the running count from the top reaches rem
@@ -413,10 +503,11 @@ __global__ void __launch_bounds__(BS_THREADS, 1) select_kernel(const SelectArgs 
   const uint32_t ut = kmin + prefix;
   const uint32_t need = rem;  // keys equal to ut to take, 1..count(ut)
 
-  // compaction in index order: warp w walks its contiguous segment 32
-  // tokens at a time (coalesced); pass A counts, pass B writes
-  const int seg = (L + BS_WARPS - 1) / BS_WARPS;
-  const int j0 = min(L, warp * seg), j1 = min(L, j0 + seg);
+  // compaction in index order: warp w of the CTA walks its contiguous
+  // segment of the CTA's keys 32 at a time (coalesced); pass A counts,
+  // pass B writes
+  const int seg = (n + BS_WARPS - 1) / BS_WARPS;
+  const int j0 = c0 + min(n, warp * seg), j1 = c0 + min(n, warp * seg + seg);
   // keys of the warp's segment, BS_BATCH steps of 32 loaded at a time
   auto seg_keys = [&](int jb, uint32_t (&u)[BS_BATCH]) {
     float v[BS_BATCH];
@@ -426,7 +517,7 @@ __global__ void __launch_bounds__(BS_THREADS, 1) select_kernel(const SelectArgs 
       v[t] = j < j1 ? __ldg(sc + j) : 0.f;
     }
 #pragma unroll
-    for (int t = 0; t < BS_BATCH; ++t) u[t] = select_key(v[t], jb + t * 32 + lane, first_forced, bad);
+    for (int t = 0; t < BS_BATCH; ++t) u[t] = key_at(jb + t * 32 + lane, v[t]);
   };
   uint32_t gt = 0, eq = 0;
   for (int jb = j0; jb < j1; jb += 32 * BS_BATCH) {
@@ -444,7 +535,24 @@ __global__ void __launch_bounds__(BS_THREADS, 1) select_kernel(const SelectArgs 
     w_eq[warp] = eq;
   }
   __syncthreads();
-  if (warp == 0) {   // per-warp bases: ties go to the earlier warps first
+  if (warp == 0) {   // this CTA's totals, published for the later ranks
+    uint32_t g = w_gt[lane], e = w_eq[lane];
+    g = __reduce_add_sync(0xffffffffu, g);
+    e = __reduce_add_sync(0xffffffffu, e);
+    if (lane == 0) {
+      s_gt = g;
+      s_eq = e;
+    }
+  }
+  cluster_sync();
+  if (warp == 0) {   // per-warp bases: ties go to the earlier ranks and warps first
+    uint32_t eq_before = 0, base = 0;
+    for (uint32_t rk = 0; rk < crank; ++rk) {
+      const uint32_t g = ld_cluster_u32(cluster_map(smem_u32(&s_gt), rk));
+      const uint32_t e = ld_cluster_u32(cluster_map(smem_u32(&s_eq), rk));
+      base += g + (need > eq_before ? min(e, need - eq_before) : 0u);
+      eq_before += e;
+    }
     const uint32_t e = w_eq[lane], g = w_gt[lane];
     uint32_t ei = e;
 #pragma unroll
@@ -452,7 +560,7 @@ __global__ void __launch_bounds__(BS_THREADS, 1) select_kernel(const SelectArgs 
       const uint32_t y = __shfl_up_sync(0xffffffffu, ei, o);
       if (lane >= o) ei += y;
     }
-    const uint32_t eb = ei - e;                       // ties in earlier warps
+    const uint32_t eb = eq_before + ei - e;           // ties in earlier ranks and warps
     const uint32_t te = need > eb ? min(e, need - eb) : 0u;
     const uint32_t t = g + te;
     uint32_t ti = t;
@@ -461,7 +569,7 @@ __global__ void __launch_bounds__(BS_THREADS, 1) select_kernel(const SelectArgs 
       const uint32_t y = __shfl_up_sync(0xffffffffu, ti, o);
       if (lane >= o) ti += y;
     }
-    w_base[lane] = ti - t;
+    w_base[lane] = base + ti - t;
     w_eqb[lane] = eb;
   }
   __syncthreads();
@@ -482,7 +590,8 @@ __global__ void __launch_bounds__(BS_THREADS, 1) select_kernel(const SelectArgs 
       eq_seen += __popc(eqm);
     }
   }
-  for (int i = k + threadIdx.x; i < cap; i += BS_THREADS) out[i] = -1;
+  for (int i = max(k, o0) + threadIdx.x; i < o1; i += BS_THREADS) out[i] = -1;
+  cluster_sync();   // no CTA leaves while another may still read its shared memory
 }
 
 }  // namespace tsa

@@ -34,8 +34,9 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 // Proxy-score work split (see score.cuh): each head's window padded to a
 // multiple of 32 rows, as many query heads of a KV group per CTA as fit in
-// 512 packed rows, and key chunks sized so the grid is about two waves of
-// 148 SMs (one CTA per SM), never below 4 key tiles.
+// 512 packed rows, and key chunks sized so the grid is one wave of 148 SMs
+// (one CTA per SM), never below 16 key tiles: a CTA loads its packed query
+// rows once, so short chunks would spend their time reloading them.
 struct ScorePlan {
   int W32, GH, n_hg, n_rp, MT, chunk_tiles, n_chunks;
 };
@@ -51,7 +52,7 @@ ScorePlan score_plan(const tsa_params* p) {
   s.MT = s.n_rp > 1 ? tsa::SC_MAX_MT : (rows + 127) / 128;
   const int tiles = (p->L + tsa::SC_KEYS - 1) / tsa::SC_KEYS;
   const int ctas = p->B * p->Hkv * s.n_hg;
-  const int per = std::max(1, (2 * 148) / ctas);
+  const int per = std::max(1, 148 / ctas);
   s.chunk_tiles = std::max(tsa::SC_MIN_CHUNK_TILES, (tiles + per - 1) / per);
   const int span = s.chunk_tiles * tsa::SC_KEYS;
   s.n_chunks = (p->L + span - 1) / span;
@@ -284,7 +285,7 @@ tsa_status run_budget(const tsa_params* p, const float* scores, int32_t* k_head,
                       uint32_t* status, cudaStream_t st, bool partial = false) {
   if (!ensure_smem(g_budget, tsa::budget_kernel, kBudgetSmem)) return TSA_ERR_CUDA;
   tsa::BudgetArgs a{scores, k_head, status, p->L, p->Hq, p->keep_recent, static_cast<double>(p->tau), seqs_of(p)};
-  tsa::budget_kernel<<<p->B * p->Hq, tsa::BS_THREADS, kBudgetSmem, st>>>(a);
+  tsa::budget_kernel<<<p->B * p->Hq * tsa::BS_CLUSTER, tsa::BS_THREADS, kBudgetSmem, st>>>(a);
   const bool mean = p->budget_mode == TSA_BUDGET_MEAN;
   if (k_seq) tsa::budget_finalize_kernel<<<p->B, 32, 0, st>>>(k_head, k_seq, p->Hq, mean ? (partial ? 2 : 1) : 0);
   return launch_ok();
@@ -294,7 +295,7 @@ tsa_status run_select(const tsa_params* p, const float* scores, const int32_t* k
                       cudaStream_t st) {
   if (!ensure_smem(g_select, tsa::select_kernel, kSelectSmem)) return TSA_ERR_CUDA;
   tsa::SelectArgs a{scores, kept_of(p, kept), idx, p->L, p->Hq, p->keep_recent, seqs_of(p)};
-  tsa::select_kernel<<<p->B * p->Hq, tsa::BS_THREADS, kSelectSmem, st>>>(a);
+  tsa::select_kernel<<<p->B * p->Hq * tsa::BS_CLUSTER, tsa::BS_THREADS, kSelectSmem, st>>>(a);
   return launch_ok();
 }
 
