@@ -45,12 +45,17 @@ ScorePlan score_plan(const tsa_params* p) {
   ScorePlan s;
   const int G = p->Hq / p->Hkv;
   s.W32 = (p->w + 31) / 32 * 32;
+  const int tiles = (p->L + tsa::SC_KEYS - 1) / tsa::SC_KEYS;
+  const int max_chunks = std::max(1, tiles / tsa::SC_MIN_CHUNK_TILES);
+  // the most heads per CTA that fit, halved while a grid of such CTAs
+  // (keys split no finer than SC_MIN_CHUNK_TILES) leaves SMs idle: short
+  // sequences gain more from parallel heads than from sharing K tiles
   s.GH = s.W32 <= tsa::SC_PASS_ROWS ? std::min(G, tsa::SC_PASS_ROWS / s.W32) : 1;
+  while (s.GH > 1 && p->B * p->Hkv * ((G + s.GH - 1) / s.GH) * max_chunks < 148) s.GH = (s.GH + 1) / 2;
   s.n_hg = (G + s.GH - 1) / s.GH;
   const int rows = s.GH * s.W32;
   s.n_rp = (rows + tsa::SC_PASS_ROWS - 1) / tsa::SC_PASS_ROWS;
   s.MT = s.n_rp > 1 ? tsa::SC_MAX_MT : (rows + 127) / 128;
-  const int tiles = (p->L + tsa::SC_KEYS - 1) / tsa::SC_KEYS;
   const int ctas = p->B * p->Hkv * s.n_hg;
   const int per = std::max(1, 148 / ctas);
   s.chunk_tiles = std::max(tsa::SC_MIN_CHUNK_TILES, (tiles + per - 1) / per);
