@@ -26,6 +26,10 @@ namespace tsa {
 // Pairs e (of the 16 value pairs of each 32-column chunk of a softmax row)
 // whose two exponentials are computed by exp2_poly_x2 on the FMA pipe; the
 // others use ex2.approx on the MUFU unit.  The split balances the two units.
+#ifndef TSA_P_SPLITS
+#define TSA_P_SPLITS 2
+#endif
+
 #ifndef TSA_EXP_EMU_PAIRS
 #define TSA_EXP_EMU_PAIRS 0x0000u
 #endif
@@ -87,7 +91,7 @@ struct Attn2Layout {
   static constexpr int NCH = D / 64;
   static constexpr int TILE = 128 * D * 2;            // bytes of one Q, K or V tile
   static constexpr int NSLOT = D == 128 ? 4 : 9;      // K/V ring slots
-  static constexpr int P_SPLITS = 2;                  // P released in this many column groups
+  static constexpr int P_SPLITS = TSA_P_SPLITS;       // P released in this many column groups
   static constexpr int KSTEPS = BN / 16;              // P.V k-steps per KV tile
   static constexpr int OFF_Q0 = 0;
   static constexpr int OFF_Q1 = TILE;
@@ -451,9 +455,8 @@ __global__ void __launch_bounds__(Attn2Layout<D>::THREADS, 1)
       // is already in registers, so P may overwrite any S column.  The plain
       // kernel stores a group's P (its two chunks, 32 columns) in one go; the
       // scatter and block-mask variants (more registers live) chunk by chunk.
-      constexpr bool kWide = !kScatter && !kBlocks;
       constexpr int CPG = 4 / C::P_SPLITS;          // 32-column chunks per P group
-      static_assert(CPG == 2, "one 32-column P store per group");
+      constexpr bool kWide = !kScatter && !kBlocks && CPG == 2;
 #pragma unroll
       for (int g = 0; g < C::P_SPLITS; ++g) {
         uint32_t pk32[32];
@@ -491,14 +494,27 @@ __global__ void __launch_bounds__(Attn2Layout<D>::THREADS, 1)
           if (pc > 0 && __any_sync(0xffffffffu, resc)) {
             if (!(live = __all_sync(0xffffffffu, mbar_wait(bar(C::B_PV + tt), (pc - 1) & 1, wc)))) break;
             tc_fence_after();
+            if constexpr (C::P_SPLITS == 2) {
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-              float ov[32];
-              tmem_ld32(o_col + c * 32, ov);
-              tmem_ld_wait();
+              for (int c = 0; c < D / 32; ++c) {
+                float ov[32];
+                tmem_ld32(o_col + c * 32, ov);
+                tmem_ld_wait();
 #pragma unroll
-              for (int e = 0; e < 32; ++e) ov[e] *= alpha;
-              tmem_st32(o_col + c * 32, ov);
+                for (int e = 0; e < 32; ++e) ov[e] *= alpha;
+                tmem_st32(o_col + c * 32, ov);
+              }
+            } else {  // more S values still live at group 0: 16 columns at a time
+#pragma unroll
+              for (int c = 0; c < D / 16; ++c) {
+                float ov[16];
+                tmem_ld16(o_col + c * 16, ov);
+                tmem_ld_wait();
+                uint32_t ou[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) ou[e] = __float_as_uint(ov[e] * alpha);
+                tmem_st16u(o_col + c * 16, ou);
+              }
             }
           }
           if (diag && last_active && (j * C::BN + C::BN > valid)) {
