@@ -434,13 +434,13 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
     import token_sparse_attention_tsa_b200 as T
 
     dist = None
-    if world > 1:
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:   # the device is set first, so NCCL binds each rank to its own GPU
         import datetime
         import torch.distributed as dist_mod
         dist = dist_mod
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
     T.load()
     stream = torch.cuda.current_stream()
 
@@ -495,7 +495,7 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
     # the kernels tsa_forward runs, one ABI call each (with head sharding, the
     # budget's all-reduce over the ranks between the budget and the selection)
     exchange_op = T.budget_reduce_op(args.budget_mode) if sharded else None
-    stage_names = ["score", "budget"] + (["exchange"] if exchange_op == "max" else []) + \
+    stage_names = ["score", "budget"] + (["exchange"] if exchange_op is not None else []) + \
         ["select", "gather", "attend", "scatter"]
 
     def staged(evs):
@@ -507,6 +507,11 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
         evs[next(n)].record(stream)
         if exchange_op == "max":
             dist.all_reduce(k_seq, op=dist.ReduceOp.MAX)
+            evs[next(n)].record(stream)
+        elif exchange_op == "sum":    # mean budget: the heads' counts summed over the ranks, as tsa_forward_end
+            tot = k_head.sum(dim=1, dtype=torch.int64)
+            dist.all_reduce(tot, op=dist.ReduceOp.SUM)
+            k_seq.copy_(torch.div(tot + wl_all.Hq - 1, wl_all.Hq, rounding_mode="floor").to(torch.int32))
             evs[next(n)].record(stream)
         T.tsa_select(p, scores, kept, idx, ws)
         evs[next(n)].record(stream)
