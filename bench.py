@@ -434,13 +434,17 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
     import token_sparse_attention_tsa_b200 as T
 
     dist = None
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
+    # one rank per GPU; with fewer GPUs than ranks (a test of the sharded
+    # path's plumbing only) ranks share devices round-robin
+    dev = torch.device("cuda", local_rank % torch.cuda.device_count())
+    torch.cuda.set_device(dev)
     if world > 1:   # the device is set first, so NCCL binds each rank to its own GPU
         import datetime
         import torch.distributed as dist_mod
         dist = dist_mod
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+        backend = os.environ.get("TSA_BENCH_BACKEND", "nccl")   # gloo: host-side exchange, for plumbing tests
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=300),
+                                device_id=dev if backend == "nccl" else None)
     T.load()
     stream = torch.cuda.current_stream()
 
@@ -551,7 +555,7 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
     torch.cuda.synchronize()
 
     # ---- headline: tsa_forward, inputs resident in HBM (all > L2)
-    with ClockSampler(local_rank) as clk:
+    with ClockSampler(dev.index) as clk:
         ms = timed(forward, args.steps)
     clocks = clk.summary()
     kept_np = kept.cpu().numpy()
