@@ -526,17 +526,23 @@ def run_gpu(args, wl, rank: int, world: int, local_rank: int) -> int:
         T.tsa_scatter(p, qc, idx, kept, o, ws)
         evs[next(n)].record(stream)
 
-    # the stage calls tsa_forward does not use, timed for comparison: the
+    # the stage calls tsa_forward does not use, timed for comparison next to
+    # the pair it does use (attention into a compressed output, then the
+    # scatter), in the same iterations so that all see the same clocks: the
     # attention with the scatter folded into its epilogue (plus the zero fill
     # of the unselected rows), and the variant that also gathers by index
-    unfused_names = ["attend_scatter_fused", "attend_gathered"]
+    unfused_names = ["attend_then_scatter", "attend_scatter_fused", "attend_gathered"]
+    oc = torch.empty_like(qc)
 
     def unfused(evs):
         evs[0].record(stream)
-        T.tsa_attend_scatter(p, qc, kc, vc, idx, kept, o, None, ws)
+        T.tsa_attend(p, qc, kc, vc, kept, oc, None, ws)
+        T.tsa_scatter(p, oc, idx, kept, o, ws)
         evs[1].record(stream)
-        T.tsa_attend_gathered(p, q, k, v, idx, kept, o, None, ws)
+        T.tsa_attend_scatter(p, qc, kc, vc, idx, kept, o, None, ws)
         evs[2].record(stream)
+        T.tsa_attend_gathered(p, q, k, v, idx, kept, o, None, ws)
+        evs[3].record(stream)
 
     def timed(fn, n):
         barrier()
