@@ -233,13 +233,28 @@ def oracle_sample(wl, tau: float, rows: int = 1536, heads: int = 2, keep_recent:
                        f"step 5 by causal pair count, to the full step ({sample_seconds:.1f} s measured)")}
 
 
+L2_BYTES = 126 << 20   # B200 L2
+
+
+def l2_note(wl) -> str:
+    """Whether the step's inputs exceed L2 (the timing rule between timed
+    iterations: flush L2 or use inputs larger than it), with their sizes."""
+    q = wl.B * wl.Hq * wl.L * wl.d * 2
+    kv = wl.B * wl.Hkv * wl.L * wl.d * 2
+    mib = lambda n: f"{n / 2**30:.3g} GiB" if n >= 2**30 else f"{n / 2**20:.3g} MiB"
+    sizes = f"Q {mib(q)}, K/V {mib(kv)} each"
+    if q + 2 * kv > L2_BYTES:
+        return f"inputs larger than L2 ({sizes})"
+    return f"inputs fit in L2 ({sizes}): a small case, not a headline timing"
+
+
 def config_of(args, wl, world: int) -> dict:
     """The workload description both arms print."""
     shard = getattr(args, "shard", "heads")
     return {"workload": wl.name, "B": wl.B, "Hq": wl.Hq, "Hkv": wl.Hkv, "L": wl.L, "d": wl.d, "w": wl.w,
             "tau": args.tau, "budget_mode": args.budget_mode, "keep_recent": args.keep_recent,
             "layout": args.layout, "parallelism": f"{shard}{world}" if world > 1 else "single",
-            "l2": "inputs larger than L2 (Q 1 GiB, K/V 256 MiB each)"}
+            "l2": l2_note(wl)}
 
 
 def run_reference(args, wl, rank: int) -> int:
