@@ -1,9 +1,12 @@
-"""The bench's reference arm (the CPU oracle, timed on a bounded sample) runs
-on the host and prints the one JSON line the timing contract asks for."""
+"""The bench prints the one JSON line the timing contract asks for: the
+reference arm (the CPU oracle, timed on a bounded sample, on the host) and,
+on a GPU, the kernels' arm."""
 import json
 import os
 import subprocess
 import sys
+
+import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -40,3 +43,27 @@ def test_reference_arm_prints_one_contract_line():
 
 def test_reference_arm_is_rank_zero_only():
     assert _run({"RANK": "1", "WORLD_SIZE": "2"}) == []
+
+
+@pytest.mark.gpu
+def test_gpu_arm_line_has_every_contract_key():
+    out = subprocess.run(
+        [sys.executable, os.path.join(ROOT, "bench.py"), "--workload", "c1_L1K_mha_d64", "--steps", "2",
+         "--warmup", "3", "--no-cpu-baseline"],
+        cwd=ROOT, capture_output=True, text=True, timeout=900)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [l for l in out.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "roofline", "e2e", "gpu_launches", "clocks",
+                "stage_ms", "unfused_stage_ms", "k_seq"):
+        assert key in d, key
+    assert d["value"] > 0 and d["steps"] == 2 and d["warmup"] == 3 and d["dtype"] == "bf16"
+    assert d["gpu_launches"] == 9 * d["steps"]
+    roof = d["roofline"]
+    assert roof["bound"] == "tensor" and roof["unit"] == "TFLOP/s" and roof["achieved"] > 0 and roof["peak"] > 0
+    assert abs(roof["frac"] - roof["achieved"] / roof["peak"]) < 1e-9
+    e2e = d["e2e"]
+    assert e2e["value"] > 0 and e2e["h2d_bytes_per_step"] > 0 and e2e["d2h_bytes_per_step"] > 0
+    assert set(d["unfused_stage_ms"]) == {"attend_then_scatter", "attend_scatter_fused", "attend_gathered"}
